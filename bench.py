@@ -1,0 +1,382 @@
+#!/usr/bin/env python3
+"""Benchmark: SAGA + Atop-N decode attention, microseconds per decode step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl ours|reference]
+
+A step is one decode token of the Atop-N loop: refresh (exact radix select of
+the N-th largest logit) when t mod n == 0, otherwise the fused reuse step,
+always followed by the kept-entry softmax and gathered value sum.  Warm-up
+runs steps 0..W-1; the timed region runs steps W..W+K-1 as one CUDA-graph
+replay ("compiled CUDA graphs", as in the pages' latency protocol), timed
+with CUDA events on the capture stream, max over ranks.  Inputs (K and V
+caches of 3 GB at the default workload) are larger than the 126 MB L2, so
+no flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  N > 1 runs independent replicas (one batch
+per GPU, no collective on the data path; weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+from sparse_decode_attention_saga_b200.workload import CONFIGS, bf16_bits, make_cache, make_queries
+
+DEFAULT_CONFIG = "llama_b16_128k"
+METRIC = "Atop-N SAGA decode attn µs/step, HBM GB/s (% peak) at 128K ctx, batch 1/16"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=320)   # 10 runs x 32 tokens
+    ap.add_argument("--warmup", type=int, default=32)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+        0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons = [], set()
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nvml:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nvml:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample_us_per_step(w, seed, steps_sample, t0):
+    """Times the CPU oracle on one batch element for `steps_sample` steps
+    starting at step t0 (refresh steps included as the schedule says) and
+    scales to the whole batch.  Returns (us_per_step, cores, description)."""
+    import oracle  # test infrastructure: only this leg of the benchmark runs it
+    ws = w.scaled(batch=1)
+    K, V = make_cache(ws, seed)
+    qs = make_queries(ws, seed, steps=t0 + steps_sample)
+    Kh, Vh = bf16_bits(K), bf16_bits(V)
+    tau = np.full((1, w.h_q), np.nan, np.float32)
+    # state entering t0: refresh at the last multiple of n before t0
+    t_last = (t0 // w.n) * w.n
+    oracle.atopn_step(bf16_bits(qs[t_last]), Kh, Vh, tau, w.N, t_last, w.n)
+    times = []
+    for t in range(t0, t0 + steps_sample):
+        a = time.perf_counter()
+        oracle.atopn_step(bf16_bits(qs[t]), Kh, Vh, tau, w.N, t, w.n)
+        times.append(time.perf_counter() - a)
+    us = float(np.mean(times)) * 1e6 * w.batch
+    desc = (f"oracle steps {t0}..{t0 + steps_sample - 1} on 1 of {w.batch} batch elements "
+            f"(all {w.h_q} query heads, l_kv={w.l_kv}), scaled x{w.batch}")
+    return us, oracle.num_threads(), desc
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = CONFIGS[args.config]
+    n_sample = max(1, args.steps)
+    # bounded: one batch element per step, at most 64 sampled steps
+    n_sample = min(n_sample, 64)
+    us, cores, desc = oracle_sample_us_per_step(w, args.seed, n_sample, args.warmup)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "us/step",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_k": w.h_k,
+                   "h_v": w.h_v, "head_dim": w.head_dim, "l_kv": w.l_kv, "N": w.N, "n": w.n,
+                   "parallelism": "replicas" if args.gpus > 1 else "single"},
+        "cpu_baseline": {"value": us, "unit": "us/step", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+
+def distinct_value_rows(idx, cnt, w):
+    """Distinct (batch, value head, position) rows kept by any query head."""
+    b, hq, l = w.batch, w.h_q, w.l_kv
+    vh = torch.arange(hq, device="cuda") * w.h_v // hq
+    valid = torch.arange(l, device="cuda")[None, None, :] < cnt[..., None]
+    rows = torch.zeros(b, w.h_v, l, dtype=torch.bool, device="cuda")
+    bi = torch.arange(b, device="cuda")[:, None, None].expand(b, hq, l)
+    vi = vh[None, :, None].expand(b, hq, l)
+    pi = idx.long().clamp(min=0)
+    rows[bi[valid], vi[valid], pi[valid]] = True
+    return int(rows.sum().item()), int(cnt.sum().item())
+
+
+def run_ours(args, world, rank, local):
+    from sparse_decode_attention_saga_b200 import _lib
+    from sparse_decode_attention_saga_b200.decoder import AtopNDecoder
+
+    w = CONFIGS[args.config]
+    seed = args.seed + rank
+    total_steps = args.warmup + args.steps
+    K, V = make_cache(w, seed, "cuda")
+    qs = make_queries(w, seed, "cuda", steps=total_steps)
+    dec = AtopNDecoder.for_workload(w)
+    stream = torch.cuda.Stream()
+    launches0 = _lib.launch_count()
+
+    with torch.cuda.stream(stream):
+        # warm-up (eager), steps 0..W-1; also caches device properties
+        for t in range(args.warmup):
+            dec.step(t, qs[t], K, V)
+        dense_out = torch.empty_like(dec.out)
+        dec.dense(qs[0], K, V, out=dense_out)
+    stream.synchronize()
+    assert dec.error() == _lib.SAGA_OK
+
+    # capture steps W..W+K-1 as one graph
+    graph = torch.cuda.CUDAGraph()
+    before = _lib.launch_count()
+    with torch.cuda.graph(graph, stream=stream):
+        for t in range(args.warmup, total_steps):
+            dec.step(t, qs[t], K, V)
+    gpu_launches = _lib.launch_count() - before
+    refresh_steps = sum(1 for t in range(args.warmup, total_steps) if t % w.n == 0)
+
+    sampler = ClockSampler(local)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        with torch.cuda.stream(stream):   # replay, and its events, on the capture stream
+            ev0.record(stream)
+            graph.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms, world)
+    us_per_step = ms * 1e3 / args.steps
+    assert dec.error() == _lib.SAGA_OK
+
+    # ---- separately timed step kinds (eager, events on the launching stream)
+    def time_steps(fn, reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            fn(0)
+            e0.record(stream)
+            for r in range(reps):
+                fn(r)
+            e1.record(stream)
+        stream.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / reps
+
+    reuse_t = [t for t in range(1, w.n)]
+    us_reuse = time_steps(lambda r: dec.step(reuse_t[r % len(reuse_t)], qs[reuse_t[r % len(reuse_t)]], K, V), 20)
+    us_refresh = time_steps(lambda r: dec.step(0, qs[0], K, V), 5)
+    us_dense = time_steps(lambda r: dec.dense(qs[r % 4], K, V, out=dense_out), 10)
+    us_mix = (us_refresh + (w.n - 1) * us_reuse) / w.n
+
+    # ---- dominant kernel: the fused compare kernel of the reuse step
+    kern_us = []
+    ks, ke = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ks.record(stream)
+        ke.record(stream)  # materialise the events before handing them to the library
+    stream.synchronize()
+    for r in range(20):
+        t = reuse_t[r % len(reuse_t)]
+        with torch.cuda.stream(stream):
+            _lib.set_kernel_events(ks, ke)
+            dec.step(t, qs[t], K, V)
+            _lib.set_kernel_events(None, None)
+        stream.synchronize()
+        kern_us.append(ks.elapsed_time(ke) * 1e3)
+    kern_us = float(np.mean(kern_us[2:]))
+
+    # kept entries and distinct value rows of a reuse step (measured, not timed)
+    idx = torch.empty((w.batch, w.h_q, w.l_kv), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((w.batch, w.h_q), dtype=torch.int32, device="cuda")
+    with torch.cuda.stream(stream):
+        dec.step(reuse_t[0], qs[reuse_t[0]], K, V, sel_idx=idx, sel_cnt=cnt)
+    stream.synchronize()
+    U, kept = distinct_value_rows(idx, cnt, w)
+    del idx
+
+    k_bytes = w.batch * w.l_kv * w.h_k * w.head_dim * 2
+    small = w.batch * w.h_q * (w.head_dim * 2 + 4)            # q + tau
+    kern_bytes = k_bytes + small + kept * 8                   # + kept (pos, logit) lists
+    step_ideal = k_bytes + U * w.head_dim * 2 + w.batch * w.h_q * (w.head_dim * (2 + 4) + 4)
+    peak, peak_kind = peaks()
+    achieved = kern_bytes / (kern_us * 1e-6) / 1e9
+
+    # ---- end to end through the public API with host buffers
+    q_host = qs.cpu().pin_memory()
+    out_host = torch.empty((args.steps,) + tuple(dec.out.shape), dtype=torch.float32).pin_memory()
+    q_dev = torch.empty_like(qs[0])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for k in range(args.steps):
+            t = args.warmup + k
+            q_dev.copy_(q_host[t], non_blocking=True)
+            o = dec.step(t, q_dev, K, V)
+            out_host[k].copy_(o, non_blocking=True)
+        e1.record(stream)
+    stream.synchronize()
+    barrier(world)
+    e2e_us = max_over_ranks(e0.elapsed_time(e1) * 1e3 / args.steps, world)
+
+    line = {
+        "metric": METRIC, "value": us_per_step, "unit": "us/step", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": us_per_step / 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_k": w.h_k,
+                   "h_v": w.h_v, "head_dim": w.head_dim, "l_kv": w.l_kv, "N": w.N, "n": w.n,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (K+V cache %.2f GB)" % (
+                       (K.numel() + V.numel()) * 2 / 1e9),
+                   "timing": "one CUDA-graph replay of K steps, CUDA events"},
+        "refresh_steps": refresh_steps,
+        "gpu_launches": int(gpu_launches),
+        "us_reuse_step": us_reuse, "us_refresh_step": us_refresh,
+        "us_mean_step_1_in_n": us_mix,
+        "us_dense_step": us_dense, "speedup_vs_dense": us_dense / us_per_step,
+        "kept_entries_per_step": kept, "distinct_value_rows": U,
+        "roofline": {"kernel": "qk_stream_kernel (fused compare, reuse step)", "bound": "hbm",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "bytes_per_launch": kern_bytes, "us_per_launch": kern_us,
+                     "traffic": None},
+        "step_roofline": {"what": "reuse step (fused kernel + gather + combine) vs ideal bytes "
+                                  "K + distinct kept V rows + q/tau/out",
+                          "ideal_bytes": step_ideal, "us": us_reuse,
+                          "achieved": step_ideal / (us_reuse * 1e-6) / 1e9,
+                          "frac": step_ideal / (us_reuse * 1e-6) / 1e9 / peak},
+        "e2e": {"value": e2e_us, "unit": "us/step",
+                "h2d_bytes_per_step": int(qs[0].numel() * 2),
+                "d2h_bytes_per_step": int(dec.out.numel() * 4)},
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        us_cpu, cores, desc = oracle_sample_us_per_step(w, args.seed, 2, w.n - 1)
+        line["cpu_baseline"] = {"value": us_cpu, "unit": "us/step", "cores": cores,
+                                "kind": "oracle", "sample": desc}
+    del graph
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

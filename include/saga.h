@@ -1,0 +1,159 @@
+/*
+ * saga.h - C ABI of the SAGA + Atop-N single-token decode attention library
+ * (libsaga.so, hand-written CUDA for sm_100a).
+ *
+ * Method: "More Value per Key: Asymmetric Sparse Attention for Faster LLM
+ * Decoding" (arXiv 2610.04753).  SAGA decouples the key-head count h_k from
+ * the value-head count h_v (ai.info summary, Key Contributions #3); Atop-N
+ * keeps, per (batch, query head), the cached positions whose logit is >= a
+ * threshold that is the exact N-th largest logit, recomputed only every n
+ * decode steps and reused in between, found by per-element comparison
+ * instead of sorting (Key Contributions #2, Methodology in Plain English
+ * ¶2); the probability-value product then touches only the kept value rows
+ * (Main Findings, "Bottleneck shift").
+ *
+ * Shapes and layouts (all row-major, innermost last; bf16 = IEEE bfloat16):
+ *   q      [batch, h_q, head_dim]            bf16   this step's queries
+ *   k      [batch, l_cap, h_k, head_dim]     bf16   key cache
+ *   v      [batch, l_cap, h_v, head_dim]     bf16   value cache
+ *          positions 0 .. l_kv-1 of each batch element are valid; rows
+ *          l_kv .. l_cap-1 are capacity and are never used.
+ *   logits [batch, h_q, l_kv]                fp32   s = q.k / sqrt(head_dim)
+ *   thresh [batch, h_q]                      fp32   Atop-N thresholds (tau)
+ *   out    [batch, h_q, head_dim]            fp32
+ *   sel_idx[batch, h_q, l_kv]                int32  kept positions, ascending,
+ *                                                   first sel_cnt entries valid
+ *   sel_cnt[batch, h_q]                      int32
+ * Head maps: query head i reads key head i*h_k/h_q and value head i*h_v/h_q
+ * (contiguous groups, as in grouped-query attention).
+ *
+ * Supported shapes: head_dim in {64, 128}; h_k in {1, 2, 4, 8}; h_q a
+ * multiple of h_k and of h_v with h_q/h_k <= 16 and h_q <= 128;
+ * saga_decode_dense also needs h_v <= 2*h_k; 1 <= l_kv <= l_cap;
+ * batch*l_cap < 2^31.  Others return SAGA_ERR_UNSUPPORTED.
+ *
+ * Conventions shared by every call:
+ *   - Ownership: the caller allocates and owns every buffer (device memory,
+ *     16-byte aligned), the thresholds and the workspace included.  The
+ *     library allocates no device memory.
+ *   - Asynchrony: every call only enqueues work on `stream` and returns; no
+ *     call synchronises the host or reads device data back.  All grids are
+ *     sized from the shapes, never from data, so a sequence of calls can be
+ *     captured in a CUDA graph (make one uncaptured call per shape first so
+ *     device properties are cached outside the capture).
+ *   - Validation: arguments are checked before anything is enqueued; on an
+ *     error nothing is launched and no output is touched.
+ *   - Workspace: `ws` must hold saga_workspace_bytes(dims, N) bytes and must
+ *     be zeroed once after allocation (or passed to saga_workspace_reset).
+ *     Calls that share a workspace must be ordered on one stream.
+ *   - Device-side faults: kernels bound every wait; a wait that runs out
+ *     sets a sticky flag in the workspace that saga_workspace_error reads.
+ *   - Return value: SAGA_OK (0) or a negative saga_status.
+ */
+#ifndef SAGA_H
+#define SAGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st* saga_stream_t;
+
+typedef struct {
+    int32_t batch;     /* b                                   */
+    int32_t h_q;       /* query heads                          */
+    int32_t h_k;       /* key heads   (SAGA: h_k < h_v allowed) */
+    int32_t h_v;       /* value heads                          */
+    int32_t head_dim;  /* d, shared by keys and values         */
+    int32_t l_kv;      /* valid cached positions               */
+    int32_t l_cap;     /* cache capacity (row stride in positions) */
+} saga_dims;
+
+typedef enum {
+    SAGA_OK = 0,
+    SAGA_ERR_INVALID_ARG = -1,  /* null/misaligned pointer, non-positive size, l_kv > l_cap, N <= 0 */
+    SAGA_ERR_UNSUPPORTED = -2,  /* shape outside the supported set above */
+    SAGA_ERR_WORKSPACE = -3,    /* ws_bytes < saga_workspace_bytes(...) */
+    SAGA_ERR_CUDA = -4,         /* a CUDA call or launch failed */
+    SAGA_ERR_DEVICE = -5,       /* no device, or the device is not sm_100 */
+    SAGA_ERR_TIMEOUT = -6       /* saga_workspace_error: a bounded device wait ran out */
+} saga_status;
+
+/* Bytes of workspace the calls below need for these dimensions.  Depends on
+ * the shapes only (not on N, which is checked to be positive); returns 0 for
+ * invalid or unsupported dimensions.  Host-only, no CUDA call. */
+size_t saga_workspace_bytes(const saga_dims* dims, int32_t N);
+
+/* Dense (full-attention) grouped-query decode: every cached position kept.
+ * The speedup denominator ("baseline full attention", ai.info summary, Main
+ * Findings, end-to-end speedups).  out[b,i,:] = softmax_j(s[b,i,j]) V[b,j,vh(i),:].
+ * Split-K over l_kv (flash-decoding) followed by a log-sum-exp combine. */
+int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const void* v,
+                      float* out, void* ws, size_t ws_bytes, saga_stream_t stream);
+
+/* Threshold refresh, run on steps with t mod n == 0 (the caller schedules).
+ * thresh_out[b,i] = the exact N-th largest logit of row (b,i), counting
+ * duplicates (Key Contributions #2: "exact top-N thresholds computed once
+ * every n tokens"); N >= l_kv gives -inf (keep everything); a threshold of
+ * -0.0 is written as +0.0.
+ *   logits_in  != NULL: use these logits [b,h_q,l_kv]; q and k are ignored.
+ *   logits_in  == NULL: compute the logits from q and k; if logits_out is
+ *                       not NULL they are also written there, so the
+ *                       following saga_atopn_decode can reuse them.
+ * Exact radix select (three passes over 32-bit order-preserving keys). */
+int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const void* k,
+                      const float* logits_in, float* logits_out, float* thresh_out,
+                      void* ws, size_t ws_bytes, saga_stream_t stream);
+
+/* One Atop-N decode step with the thresholds `thresh` (fresh from
+ * saga_topn_refresh on refresh steps, reused otherwise):
+ *   tau_eff = min(thresh[b,i], max_j s[b,i,j]);  keep j  <=>  s[b,i,j] >= tau_eff;
+ *   out[b,i,:] = sum_kept softmax(s) V[b,j,vh(i),:].
+ * The min() keeps the row's maximal entries when a stale threshold lies
+ * above every logit (the pages are silent on that case).
+ *   logits_in != NULL: the logits are read from there (q, k unused); the
+ *                      select/compact, gathered-PV and combine kernels run.
+ *   logits_in == NULL and sel_idx == NULL: the fused kernel computes the
+ *                      logits on chip, compares, and gathers only the kept
+ *                      value rows; logits never reach device memory.
+ *   logits_in == NULL and sel_idx != NULL: logits go through the workspace
+ *                      so the kept positions can be emitted.
+ * sel_idx (nullable): kept positions of each row, ascending.
+ * sel_cnt (nullable): number kept per row. */
+int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const void* v,
+                      const float* thresh, const float* logits_in, float* out,
+                      int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
+                      saga_stream_t stream);
+
+/* Enqueue a zeroing of the workspace (sticky flags included). */
+int saga_workspace_reset(void* ws, size_t ws_bytes, saga_stream_t stream);
+
+/* Synchronise `stream`, read and clear the workspace's sticky device flag:
+ * SAGA_OK, SAGA_ERR_TIMEOUT, or SAGA_ERR_CUDA if the read itself failed. */
+int saga_workspace_error(void* ws, size_t ws_bytes, saga_stream_t stream);
+
+/* Static description of a status code. */
+const char* saga_status_string(int status);
+
+/* Number of kernels this library has launched in this process (host counter,
+ * incremented per launch; graph replays are not counted). */
+uint64_t saga_launch_count(void);
+
+/* Measurement hook for the calling host thread: while set, the dominant
+ * kernel of each call (the fused decode kernel, the dense kernel, the logits
+ * kernel) is bracketed by cudaEventRecord(start) / cudaEventRecord(stop) on
+ * the call's stream.  Pass NULL, NULL to clear.  Events are cudaEvent_t. */
+void saga_set_kernel_events(void* start_event, void* stop_event);
+
+/* ABI version (major * 100 + minor). */
+int saga_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGA_H */

@@ -1,0 +1,156 @@
+"""ctypes binding of ``libsaga.so`` (include/saga.h): argument marshalling only.
+
+Every function here forwards to the C entry point of the same name, passing
+device pointers (``tensor.data_ptr()``) and the current CUDA stream; all work
+runs in the library's kernels.  A missing library raises immediately: there
+is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_HERE, "libsaga.so")
+
+SAGA_OK = 0
+SAGA_ERR_INVALID_ARG = -1
+SAGA_ERR_UNSUPPORTED = -2
+SAGA_ERR_WORKSPACE = -3
+SAGA_ERR_CUDA = -4
+SAGA_ERR_DEVICE = -5
+SAGA_ERR_TIMEOUT = -6
+
+EXPORTS = (
+    "saga_workspace_bytes", "saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
+    "saga_workspace_reset", "saga_workspace_error", "saga_status_string", "saga_launch_count",
+    "saga_set_kernel_events", "saga_version",
+)
+
+
+class SagaDims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_k", ctypes.c_int32),
+                ("h_v", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("l_kv", ctypes.c_int32),
+                ("l_cap", ctypes.c_int32)]
+
+
+class SagaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+_path = LIBRARY
+
+
+def load(path: str | None = None):
+    """Loads the library (once); raises if it has not been built."""
+    global _lib, _path
+    if path is not None and path != _path:
+        _lib, _path = None, path
+    if _lib is None:
+        if not os.path.exists(_path):
+            raise RuntimeError(
+                f"{_path} is missing: build it with `python -m sparse_decode_attention_saga_b200.build` "
+                "(the CUDA library is required; there is no CPU fallback)")
+        lib = ctypes.CDLL(_path)
+        P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        D = ctypes.POINTER(SagaDims)
+        lib.saga_workspace_bytes.argtypes = [D, I32]
+        lib.saga_workspace_bytes.restype = SZ
+        lib.saga_decode_dense.argtypes = [D, P, P, P, P, P, SZ, P]
+        lib.saga_topn_refresh.argtypes = [D, I32, P, P, P, P, P, P, SZ, P]
+        lib.saga_atopn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.saga_workspace_reset.argtypes = [P, SZ, P]
+        lib.saga_workspace_error.argtypes = [P, SZ, P]
+        lib.saga_status_string.argtypes = [ctypes.c_int]
+        lib.saga_status_string.restype = ctypes.c_char_p
+        lib.saga_launch_count.restype = ctypes.c_uint64
+        lib.saga_set_kernel_events.argtypes = [P, P]
+        lib.saga_set_kernel_events.restype = None
+        for f in ("saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
+                  "saga_workspace_reset", "saga_workspace_error", "saga_version"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, status: int) -> None:
+    if status != SAGA_OK:
+        raise SagaError(fn, status)
+
+
+def dims(batch, h_q, h_k, h_v, head_dim, l_kv, l_cap=None) -> SagaDims:
+    return SagaDims(batch, h_q, h_k, h_v, head_dim, l_kv, l_kv if l_cap is None else l_cap)
+
+
+def status_string(status: int) -> str:
+    return load().saga_status_string(int(status)).decode()
+
+
+def workspace_bytes(d: SagaDims, N: int) -> int:
+    return int(load().saga_workspace_bytes(ctypes.byref(d), int(N)))
+
+
+def decode_dense(d, q, k, v, out, ws, stream=None) -> None:
+    st = load().saga_decode_dense(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check("saga_decode_dense", st)
+
+
+def topn_refresh(d, N, q, k, logits_in, logits_out, thresh_out, ws, stream=None) -> None:
+    st = load().saga_topn_refresh(ctypes.byref(d), int(N), _ptr(q), _ptr(k), _ptr(logits_in),
+                                  _ptr(logits_out), _ptr(thresh_out), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream))
+    _check("saga_topn_refresh", st)
+
+
+def atopn_decode(d, q, k, v, thresh, logits_in, out, sel_idx, sel_cnt, ws, stream=None) -> None:
+    st = load().saga_atopn_decode(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v), _ptr(thresh),
+                                  _ptr(logits_in), _ptr(out), _ptr(sel_idx), _ptr(sel_cnt),
+                                  _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check("saga_atopn_decode", st)
+
+
+def workspace_reset(ws, stream=None) -> None:
+    _check("saga_workspace_reset",
+           load().saga_workspace_reset(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def workspace_error(ws, stream=None) -> int:
+    return int(load().saga_workspace_error(_ptr(ws), ws.numel() * ws.element_size(),
+                                           _stream(stream)))
+
+
+def launch_count() -> int:
+    return int(load().saga_launch_count())
+
+
+def set_kernel_events(start=None, stop=None) -> None:
+    """``start``/``stop`` are torch.cuda.Event objects (or None to clear)."""
+    s = None if start is None else start.cuda_event
+    e = None if stop is None else stop.cuda_event
+    load().saga_set_kernel_events(s, e)
+
+
+def version() -> int:
+    return int(load().saga_version())

@@ -1,0 +1,235 @@
+// Streaming query-key kernel over the K cache.
+//
+// Method: "More Value per Key" (ai.info summary).  Main Findings, "Bottleneck
+// shift": once the probability-value product is sparse, the query-key
+// product over every cached position is the dominant cost, so this kernel is
+// built to stream K at HBM speed.  Key Contributions #2 / Methodology ¶2:
+// selection is a per-element comparison against the stored thresholds, not a
+// sort.
+//
+// One CTA owns a contiguous range of (batch, 32 KB tile) units.  Warp 8 is
+// the producer: it issues one TMA box per (key head, 64-dim half) into a
+// multi-stage shared-memory ring (full/empty mbarriers).  Warps 0-7 consume:
+// warp w handles key head w / (8/h_k) and a fixed slice of each tile's
+// positions, computing the logits of all G query heads of that key head on
+// tensor cores (qk_tile.cuh), then
+//   kStreamLogits: stores them to the logits array (refresh steps), or
+//   kStreamSelect: compares them with the per-(batch, query head) thresholds,
+//     ballots the kept entries and appends (position, logit) to per-(row,
+//     CTA slot, warp) lists in ascending position order, and records the
+//     count and the maximum logit seen (for the empty-set fallback).
+// Logits never reach device memory on the select path.
+#include "qk_tile.cuh"
+#include "saga_kernels.h"
+
+namespace saga {
+
+namespace {
+
+
+template <int D, int NT, int MODE>
+__global__ void __launch_bounds__(kStreamThreads, 1)
+    qk_stream_kernel(const __grid_constant__ CUtensorMap kmap, const StreamArgs a) {
+    constexpr int MBW = 128 / D;
+    constexpr int DH = D / 64;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    const int stages = a.stages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(stages) * kStageBytes);
+    uint64_t* empty = full + stages;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
+
+    const Geometry& g = a.g;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const long long T = static_cast<long long>(g.b) * g.tiles;
+    const int C = a.C, c = blockIdx.x;
+    const long long t0 = cta_tile_begin(T, C, c), t1 = cta_tile_begin(T, C, c + 1);
+    const int ntile = static_cast<int>(t1 - t0);
+    const uint32_t stage0 = smem_addr(smem);
+
+    if (warp == kConsumerWarps) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            prefetch_tensor_map(&kmap);
+            int issued = 0;
+            for (int k = 0; k < ntile; ++k) {
+                const int st = k % stages;
+                if (!mbar_wait(&empty[st], ((k / stages) & 1) ^ 1, abort_flag)) break;
+                const long long t = t0 + k;
+                const int bb = static_cast<int>(t / g.tiles);
+                const int tl = static_cast<int>(t - static_cast<long long>(bb) * g.tiles);
+                const int z = bb * g.l_cap + tl * g.P;
+                mbar_arrive_expect_tx(&full[st], kStageBytes);
+                uint8_t* dst = smem + static_cast<size_t>(st) * kStageBytes;
+                for (int kh = 0; kh < g.hk; ++kh)
+                    for (int dh = 0; dh < DH; ++dh)
+                        tma_load_3d(dst + (kh * DH + dh) * g.P * 128, &kmap, &full[st], dh * 64,
+                                    kh, z);
+                issued = k + 1;
+            }
+            // Drain: the last load armed on each stage must land before exit.
+            int dummy = 0;
+            for (int k = (issued > stages ? issued - stages : 0); k < issued; ++k)
+                if (!mbar_wait(&full[k % stages], (k / stages) & 1, &dummy))
+                    raise_device_error(a.err, kErrTimeout);
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    const int kh = warp / g.WPK, sub = warp % g.WPK;
+    const int mb0 = sub * MBW;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int G = g.G;
+    const float scale = g.scale;
+
+    QFrag<D, NT> qf;
+    float tau[NT][2], mall[NT][2];
+    int cnt[NT][2];
+    int cur_bb = -1, slot = 0;
+    long long sub_base = 0;
+
+    auto begin_segment = [&](int bb) {
+        load_q_frag<D, NT>(qf, reinterpret_cast<const __nv_bfloat16*>(a.q), g.hq, G, bb, kh, lane);
+        if (MODE == kStreamSelect) {
+            const long long x0 = static_cast<long long>(bb) * g.tiles;
+            const long long s0 = t0 > x0 ? t0 : x0;
+            const long long s1 = t1 < x0 + g.tiles ? t1 : x0 + g.tiles;
+            slot = c - cta_of_tile(x0, T, C);
+            sub_base = (s0 - x0) * g.P + static_cast<long long>(sub) * (s1 - s0) * MBW * 16;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int hl = nt * 8 + 2 * tq + e;
+                    tau[nt][e] = hl < G ? __ldg(a.thresh + bb * g.hq + kh * G + hl) : kInf;
+                    mall[nt][e] = -kInf;
+                    cnt[nt][e] = 0;
+                }
+        }
+    };
+
+    auto end_segment = [&](int bb) {
+        if (MODE != kStreamSelect) return;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float m = mall[nt][e];
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                const int hl = nt * 8 + 2 * tq + e;
+                if (gq == 0 && hl < G) {
+                    const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + hl;
+                    const size_t at = (row * g.S_cap + slot) * g.WPK + sub;
+                    a.seg_cnt[at] = cnt[nt][e];
+                    a.seg_mall[at] = m;
+                }
+            }
+    };
+
+    bool ok = true;
+    for (int k = 0; k < ntile; ++k) {
+        const long long t = t0 + k;
+        const int bb = static_cast<int>(t / g.tiles);
+        const int tl = static_cast<int>(t - static_cast<long long>(bb) * g.tiles);
+        if (bb != cur_bb) {
+            if (cur_bb >= 0) end_segment(cur_bb);
+            begin_segment(bb);
+            cur_bb = bb;
+        }
+        const int st = k % stages;
+        const bool got = mbar_wait(&full[st], (k / stages) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) {
+            ok = false;
+            break;
+        }
+        float acc[MBW][NT][4];
+        qk_mma<D, NT, MBW>(stage0 + st * kStageBytes, g.P, kh, mb0, qf, acc, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+
+        const int pos0 = tl * g.P + mb0 * 16 + gq;
+#pragma unroll
+        for (int mbi = 0; mbi < MBW; ++mbi)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int pos = pos0 + mbi * 16 + 8 * h;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int hl = nt * 8 + 2 * tq + e;
+                        const bool valid = pos < g.l && hl < G;
+                        const float s = acc[mbi][nt][2 * h + e] * scale;
+                        const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + hl;
+                        if (MODE == kStreamLogits) {
+                            if (valid) a.logits[row * g.l + pos] = s;
+                        } else {
+                            if (valid) mall[nt][e] = fmaxf(mall[nt][e], s);
+                            const bool kept = valid && s >= tau[nt][e];
+                            const uint32_t ball = __ballot_sync(0xffffffffu, kept);
+                            if (ball) {
+                                const uint32_t grp = ball & (0x11111111u << tq);
+                                if (kept) {
+                                    const int off = cnt[nt][e] + __popc(grp & lanemask_lt());
+                                    const size_t at = row * g.l_pad + sub_base + off;
+                                    a.list_idx[at] = pos;
+                                    a.list_s[at] = s;
+                                }
+                                cnt[nt][e] += __popc(grp);
+                            }
+                        }
+                    }
+            }
+    }
+    if (cur_bb >= 0) end_segment(cur_bb);
+    if (!ok && lane == 0) raise_device_error(a.err, kErrTimeout);
+}
+
+template <int D, int NT, int MODE>
+cudaError_t launch_t(const CUtensorMap& kmap, const StreamArgs& a, cudaStream_t stream) {
+    const size_t smem = stream_smem_bytes(a.stages);
+    auto kern = qk_stream_kernel<D, NT, MODE>;
+    // once per instantiation, so launches inside a stream capture set nothing
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem);
+    if (attr != cudaSuccess) return attr;
+    kern<<<a.C, kStreamThreads, smem, stream>>>(kmap, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t stream_smem_bytes(int stages) {
+    return 1024 + static_cast<size_t>(stages) * kStageBytes + 2 * stages * sizeof(uint64_t) + 16;
+}
+
+cudaError_t launch_qk_stream(int mode, const CUtensorMap& kmap, const StreamArgs& a,
+                             cudaStream_t stream) {
+    const int d = a.g.d, nt = a.g.NT;
+#define SAGA_QK_CASE(D_, NT_)                                                         \
+    if (d == D_ && nt == NT_)                                                         \
+        return mode == kStreamLogits ? launch_t<D_, NT_, kStreamLogits>(kmap, a, stream) \
+                                     : launch_t<D_, NT_, kStreamSelect>(kmap, a, stream);
+    SAGA_QK_CASE(64, 1)
+    SAGA_QK_CASE(64, 2)
+    SAGA_QK_CASE(128, 1)
+    SAGA_QK_CASE(128, 2)
+#undef SAGA_QK_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace saga

@@ -1,0 +1,167 @@
+// Exact threshold refresh: the N-th largest logit of every (batch, query
+// head) row, counting duplicates.
+//
+// Method: "More Value per Key" (ai.info summary, Key Contributions #2): Atop-N
+// reuses exact top-N thresholds computed once every n tokens.  The pages do
+// not say how the exact threshold is found; this is an MSB-first radix select
+// on order-preserving 32-bit keys (digits of 11, 11 and 10 bits), which is
+// exact and needs no sort.
+//
+// Pass p, grid (chunks, rows): each CTA histograms the digit of the keys of
+// its chunk that match the prefix fixed by the earlier passes (warp-
+// aggregated shared atomics), adds its histogram to the row's global one,
+// and takes a ticket; the CTA that takes the last ticket scans the histogram
+// from the top bin, fixes the digit that holds the rank, and stores
+// (prefix, rank) for the next pass, or the threshold after the last pass.
+// No CTA waits for another.
+#include "saga_device.cuh"
+#include "saga_kernels.h"
+
+namespace saga {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kLoads = 16;
+
+// Block-wide exclusive scan of one value per thread; returns the block total.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t& excl,
+                                                         uint32_t* warp_tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) {
+        const uint32_t x = warp_tot[w];
+        before += (w < warp) ? x : 0u;
+        total += x;
+    }
+    excl = before + inc - v;
+    return total;
+}
+
+template <int PASS>
+__global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a) {
+    constexpr int shift = PASS == 0 ? 21 : (PASS == 1 ? 10 : 0);
+    constexpr int width = PASS == 2 ? 10 : 11;
+    constexpr int nb = 1 << width;
+    constexpr int per_thread = nb / kThreads;
+    constexpr int high = (shift + width) & 31;  // bits above this digit (unused in pass 0)
+
+    __shared__ uint32_t hist[nb];
+    __shared__ uint32_t warp_tot[kThreads / 32];
+    __shared__ int is_last;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long row = blockIdx.y;
+    const int chunk = blockIdx.x;
+    for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
+    const uint32_t prefix = PASS == 0 ? 0u : __ldcg(a.state + row * 2);
+    __syncthreads();
+
+    const float* src = a.logits + row * a.l;
+    const int per = (a.l + a.chunks - 1) / a.chunks;
+    const int j0 = chunk * per;
+    const int j1 = min(a.l, j0 + per);
+    // kLoads independent coalesced loads per thread per round keep enough
+    // bytes in flight to stream the logits at HBM speed.
+    for (int base = j0; base < j1; base += kLoads * kThreads) {
+        float v[kLoads];
+#pragma unroll
+        for (int k = 0; k < kLoads; ++k) {
+            const int j = base + k * kThreads + tid;
+            v[k] = j < j1 ? __ldg(src + j) : 0.f;
+        }
+#pragma unroll
+        for (int k = 0; k < kLoads; ++k) {
+            const int j = base + k * kThreads + tid;
+            const bool valid = j < j1;
+            const uint32_t key = float_to_key(v[k]);
+            const bool cand = valid && (PASS == 0 || (key >> high) == prefix);
+            const uint32_t digit = (key >> shift) & (nb - 1);
+            if (PASS == 0) {
+                // most keys are candidates: aggregate equal digits across the warp
+                const uint32_t peers = __match_any_sync(0xffffffffu, cand ? digit : 0xffffffffu);
+                if (cand && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
+            } else if (cand) {
+                atomicAdd(&hist[digit], 1u);
+            }
+        }
+    }
+    __syncthreads();
+
+    uint32_t* ghist = a.hist + (static_cast<long long>(PASS) * a.rows + row) * kRadixBins;
+    for (int i = tid; i < nb; i += kThreads)
+        if (hist[i]) atomicAdd(ghist + i, hist[i]);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = (atomicAdd(a.tickets + row, 1u) == static_cast<uint32_t>(a.chunks - 1));
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+
+    // Last CTA of the row: find the bin holding rank `rank` counted from the
+    // top.  Thread tid owns bins [nb - (tid+1)*per_thread, nb - tid*per_thread).
+    const uint32_t rank = PASS == 0 ? static_cast<uint32_t>(a.N) : __ldcg(a.state + row * 2 + 1);
+    uint32_t cnt[per_thread];
+    uint32_t sum = 0;
+    const int top = nb - tid * per_thread;  // exclusive upper bin of this thread
+#pragma unroll
+    for (int k = 0; k < per_thread; ++k) {
+        cnt[k] = __ldcg(ghist + top - 1 - k);  // descending bins
+        sum += cnt[k];
+    }
+    uint32_t excl;
+    block_exclusive_scan(sum, excl, warp_tot);
+    if (excl < rank && rank <= excl + sum) {
+        uint32_t before = excl;
+        int digit = top - 1;
+#pragma unroll
+        for (int k = 0; k < per_thread; ++k) {
+            if (before + cnt[k] >= rank) {
+                digit = top - 1 - k;
+                break;
+            }
+            before += cnt[k];
+        }
+        const uint32_t new_prefix = (prefix << width) | static_cast<uint32_t>(digit);
+        if (PASS < kRadixPasses - 1) {
+            a.state[row * 2] = new_prefix;
+            a.state[row * 2 + 1] = rank - before;
+        } else {
+            a.thresh[row] = key_to_float(new_prefix);
+        }
+    }
+    if (tid == 0) a.tickets[row] = 0u;
+}
+
+__global__ void fill_kernel(float* p, long long n, float value) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<long long>(gridDim.x) * blockDim.x)
+        p[i] = value;
+}
+
+}  // namespace
+
+cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream) {
+    const dim3 grid(a.chunks, static_cast<unsigned>(a.rows));
+    radix_pass_kernel<0><<<grid, kThreads, 0, stream>>>(a);
+    radix_pass_kernel<1><<<grid, kThreads, 0, stream>>>(a);
+    radix_pass_kernel<2><<<grid, kThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fill(float* p, long long n, float value, cudaStream_t stream) {
+    const int blocks = static_cast<int>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+    fill_kernel<<<blocks > 0 ? blocks : 1, 256, 0, stream>>>(p, n, value);
+    return cudaGetLastError();
+}
+
+}  // namespace saga

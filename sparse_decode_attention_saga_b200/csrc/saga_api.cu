@@ -1,0 +1,455 @@
+// C ABI of libsaga.so (declared in include/saga.h): argument validation,
+// workspace carving, TMA descriptor encoding and kernel dispatch.  Every
+// check happens before anything is enqueued; nothing here allocates device
+// memory or synchronises, except saga_workspace_error which is documented to.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <mutex>
+
+#include "saga.h"
+#include "saga_kernels.h"
+#include "saga_params.h"
+
+using namespace saga;
+
+namespace {
+
+constexpr int kStreamStages = 6;  // 6 x 32 KB of K in flight per SM
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_launches{0};
+thread_local cudaEvent_t t_ev_start = nullptr;
+thread_local cudaEvent_t t_ev_stop = nullptr;
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int major = 0;
+    int max_smem = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SAGA_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        cudaDeviceProp p;
+        if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return SAGA_ERR_DEVICE;
+        d.sms = p.multiProcessorCount;
+        d.major = p.major;
+        d.max_smem = static_cast<int>(p.sharedMemPerBlockOptin);
+        d.ready = true;
+    }
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return SAGA_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *out = d;
+    return d.major == 10 ? SAGA_OK : SAGA_ERR_DEVICE;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shapes -> Geometry, or a status.
+int make_geometry(const saga_dims* d, Geometry* g) {
+    if (!d) return SAGA_ERR_INVALID_ARG;
+    if (d->batch <= 0 || d->h_q <= 0 || d->h_k <= 0 || d->h_v <= 0 || d->head_dim <= 0 ||
+        d->l_kv <= 0 || d->l_cap < d->l_kv)
+        return SAGA_ERR_INVALID_ARG;
+    if (d->head_dim != 64 && d->head_dim != 128) return SAGA_ERR_UNSUPPORTED;
+    if (d->h_k != 1 && d->h_k != 2 && d->h_k != 4 && d->h_k != 8) return SAGA_ERR_UNSUPPORTED;
+    if (d->h_q % d->h_k != 0 || d->h_q % d->h_v != 0) return SAGA_ERR_UNSUPPORTED;
+    if (d->h_q / d->h_k > 16 || d->h_q > 128) return SAGA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(d->batch) * d->l_cap >= (1ll << 31)) return SAGA_ERR_UNSUPPORTED;
+    if (static_cast<long long>(d->batch) * d->h_q > 65535) return SAGA_ERR_UNSUPPORTED;
+    Geometry& x = *g;
+    x.b = d->batch;
+    x.hq = d->h_q;
+    x.hk = d->h_k;
+    x.hv = d->h_v;
+    x.d = d->head_dim;
+    x.l = d->l_kv;
+    x.l_cap = d->l_cap;
+    x.G = x.hq / x.hk;
+    x.NT = (x.G + 7) / 8;
+    x.P = kStageBytes / (x.hk * x.d * 2);
+    x.WPK = kConsumerWarps / x.hk;
+    x.MBW = 128 / x.d;
+    x.tiles = (x.l + x.P - 1) / x.P;
+    x.l_pad = x.tiles * x.P;
+    // A batch row of `tiles` tiles meets at most 2*C/b + 2 CTA ranges when
+    // C <= b*tiles (every range holds at least floor(T/C) >= T/(2C) tiles).
+    const int per_batch = 2 * ((kMaxCtas + x.b - 1) / x.b) + 2;
+    x.S_cap = per_batch < x.tiles ? per_batch : x.tiles;
+    x.rec = x.d + kRecHeader;
+    x.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(x.d)));
+    return SAGA_OK;
+}
+
+int check_ws(const Geometry& g, const void* ws, size_t ws_bytes) {
+    if (!ws || !aligned(ws, 256)) return SAGA_ERR_INVALID_ARG;
+    if (ws_bytes < workspace_layout(g).total) return SAGA_ERR_WORKSPACE;
+    return SAGA_OK;
+}
+
+template <typename T>
+T* ws_at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+int encode_cache_map(CUtensorMap* map, const void* base, const Geometry& g, int heads,
+                     bool swizzle) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(heads),
+                          static_cast<cuuint64_t>(g.b) * g.l_cap};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.d) * 2,
+                             static_cast<cuuint64_t>(heads) * g.d * 2};
+    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(g.P)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? SAGA_OK : SAGA_ERR_CUDA;
+}
+
+int max_slots(const Geometry& g, long long T, int C) {
+    int m = 0;
+    for (int bb = 0; bb < g.b; ++bb) {
+        const int s = slots_of_batch(bb, g.tiles, T, C);
+        m = s > m ? s : m;
+    }
+    return m;
+}
+
+// Grid of the streaming kernels: one CTA per SM, at most one per tile, and
+// never more partial-record slots per batch row than the workspace holds.
+int stream_ctas(const Geometry& g, const DeviceInfo& dev) {
+    const long long T = static_cast<long long>(g.b) * g.tiles;
+    long long c = dev.sms;
+    if (c > kMaxCtas) c = kMaxCtas;
+    if (c > T) c = T;
+    int C = static_cast<int>(c < 1 ? 1 : c);
+    while (C > 1 && max_slots(g, T, C) > g.S_cap) --C;
+    return C;
+}
+
+// CTAs per row of the gather kernel: about 8 per SM over all rows, never more
+// than the partial-record slots of a row.
+int gather_parts(const Geometry& g, const DeviceInfo& dev) {
+    const long long rows = static_cast<long long>(g.b) * g.hq;
+    long long parts = (8ll * dev.sms + rows - 1) / rows;
+    const long long cap = static_cast<long long>(g.S_cap) * g.WPK;
+    if (parts > cap) parts = cap;
+    return static_cast<int>(parts < 1 ? 1 : parts);
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA; }
+
+void ev_start(cudaStream_t s) {
+    if (t_ev_start) cudaEventRecord(t_ev_start, s);
+}
+void ev_stop(cudaStream_t s) {
+    if (t_ev_stop) cudaEventRecord(t_ev_stop, s);
+}
+
+// Logits of every row into `dst` [b*hq][l] (the refresh path).
+int run_logits(const Geometry& g, const DeviceInfo& dev, const void* q, const void* k, float* dst,
+               uint32_t* err, cudaStream_t s) {
+    CUtensorMap kmap;
+    int st = encode_cache_map(&kmap, k, g, g.hk, true);
+    if (st) return st;
+    StreamArgs a{};
+    a.g = g;
+    a.C = stream_ctas(g, dev);
+    a.stages = kStreamStages;
+    a.q = q;
+    a.logits = dst;
+    a.err = err;
+    ev_start(s);
+    const cudaError_t e = launch_qk_stream(kStreamLogits, kmap, a, s);
+    ev_stop(s);
+    g_launches += 1;
+    return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t saga_workspace_bytes(const saga_dims* dims, int32_t N) {
+    Geometry g;
+    if (N <= 0 || make_geometry(dims, &g) != SAGA_OK) return 0;
+    return workspace_layout(g).total;
+}
+
+int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const void* k,
+                      const float* logits_in, float* logits_out, float* thresh_out, void* ws,
+                      size_t ws_bytes, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (N <= 0 || !thresh_out || !aligned(thresh_out, 4)) return SAGA_ERR_INVALID_ARG;
+    if (logits_in) {
+        if (!aligned(logits_in, 4)) return SAGA_ERR_INVALID_ARG;
+    } else {
+        if (!q || !k || !aligned(q, 16) || !aligned(k, 16)) return SAGA_ERR_INVALID_ARG;
+        if (logits_out && !aligned(logits_out, 4)) return SAGA_ERR_INVALID_ARG;
+    }
+    if ((st = check_ws(g, ws, ws_bytes))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsLayout L = workspace_layout(g);
+    uint32_t* err = ws_at<uint32_t>(ws, L.err);
+    const long long rows = static_cast<long long>(g.b) * g.hq;
+
+    const float* logits = logits_in;
+    if (!logits) {
+        float* dst = logits_out ? logits_out : ws_at<float>(ws, L.logits);
+        if ((st = run_logits(g, dev, q, k, dst, err, s))) return st;
+        logits = dst;
+    }
+    if (N >= g.l) {
+        g_launches += 1;
+        return cuda_status(launch_fill(thresh_out, rows, -std::numeric_limits<float>::infinity(), s));
+    }
+    cudaError_t e = cudaMemsetAsync(ws_at<uint8_t>(ws, L.hist), 0, L.cnt - L.hist, s);
+    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+    RadixArgs r{};
+    r.logits = logits;
+    r.rows = rows;
+    r.l = g.l;
+    r.N = N;
+    long long chunks = (8ll * dev.sms + rows - 1) / rows;
+    const long long max_chunks = (g.l + 2047) / 2048;
+    if (chunks > max_chunks) chunks = max_chunks;
+    r.chunks = static_cast<int>(chunks < 1 ? 1 : chunks);
+    r.hist = ws_at<uint32_t>(ws, L.hist);
+    r.state = ws_at<uint32_t>(ws, L.state);
+    r.tickets = ws_at<uint32_t>(ws, L.tickets);
+    r.thresh = thresh_out;
+    r.err = err;
+    g_launches += kRadixPasses;
+    return cuda_status(launch_radix_select(r, s));
+}
+
+int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const void* v,
+                      const float* thresh, const float* logits_in, float* out, int32_t* sel_idx,
+                      int32_t* sel_cnt, void* ws, size_t ws_bytes, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (!v || !aligned(v, 16) || !thresh || !aligned(thresh, 4) || !out || !aligned(out, 4))
+        return SAGA_ERR_INVALID_ARG;
+    if (logits_in ? !aligned(logits_in, 4) : (!q || !k || !aligned(q, 16) || !aligned(k, 16)))
+        return SAGA_ERR_INVALID_ARG;
+    if ((sel_idx && !aligned(sel_idx, 4)) || (sel_cnt && !aligned(sel_cnt, 4)))
+        return SAGA_ERR_INVALID_ARG;
+    if ((st = check_ws(g, ws, ws_bytes))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsLayout L = workspace_layout(g);
+    uint32_t* err = ws_at<uint32_t>(ws, L.err);
+    const long long rows = static_cast<long long>(g.b) * g.hq;
+    float* records = ws_at<float>(ws, L.records);
+
+    if (logits_in || sel_idx) {
+        // stored logits -> compare/compact -> gathered PV -> combine
+        const float* logits = logits_in;
+        if (!logits) {
+            float* dst = ws_at<float>(ws, L.logits);
+            if ((st = run_logits(g, dev, q, k, dst, err, s))) return st;
+            logits = dst;
+        }
+        SelectArgs sa{};
+        sa.logits = logits;
+        sa.thresh = thresh;
+        sa.rows = rows;
+        sa.l = g.l;
+        sa.idx = sel_idx ? sel_idx : ws_at<int32_t>(ws, L.list_idx);
+        sa.cnt = ws_at<int32_t>(ws, L.cnt);
+        cudaError_t e = launch_select_compact(sa, s);
+        g_launches += 1;
+        if (e != cudaSuccess) return SAGA_ERR_CUDA;
+
+        GatherArgs ga{};
+        ga.g = g;
+        ga.mode = kListContiguous;
+        ga.parts = gather_parts(g, dev);
+        ga.max_lists = 1;
+        ga.v = v;
+        ga.logits = logits;
+        ga.idx = sa.idx;
+        ga.cnt = sa.cnt;
+        ga.records = records;
+        e = launch_gather_pv(ga, s);
+        g_launches += 1;
+        if (e != cudaSuccess) return SAGA_ERR_CUDA;
+
+        CombineArgs ca{};
+        ca.g = g;
+        ca.mode = kCombineParts;
+        ca.parts = ga.parts;
+        ca.records = records;
+        ca.out = out;
+        ca.sel_cnt = sel_cnt;
+        g_launches += 1;
+        return cuda_status(launch_combine(ca, s));
+    }
+
+    // fused: stream K, compare on chip, lists -> gathered PV -> combine
+    CUtensorMap kmap;
+    if ((st = encode_cache_map(&kmap, k, g, g.hk, true))) return st;
+    StreamArgs a{};
+    a.g = g;
+    a.C = stream_ctas(g, dev);
+    a.stages = kStreamStages;
+    a.q = q;
+    a.thresh = thresh;
+    a.list_idx = ws_at<int32_t>(ws, L.list_idx);
+    a.list_s = ws_at<float>(ws, L.list_s);
+    a.seg_cnt = ws_at<int32_t>(ws, L.seg_cnt);
+    a.seg_mall = ws_at<float>(ws, L.seg_mall);
+    a.err = err;
+    ev_start(s);
+    cudaError_t e = launch_qk_stream(kStreamSelect, kmap, a, s);
+    ev_stop(s);
+    g_launches += 1;
+    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+
+    GatherArgs ga{};
+    ga.g = g;
+    ga.mode = kListSegments;
+    ga.C = a.C;
+    ga.parts = gather_parts(g, dev);
+    ga.max_lists = max_slots(g, static_cast<long long>(g.b) * g.tiles, a.C) * g.WPK;
+    if (gather_smem_bytes(ga.max_lists) > static_cast<size_t>(kGatherMaxSmem))
+        return SAGA_ERR_UNSUPPORTED;
+    ga.v = v;
+    ga.list_idx = a.list_idx;
+    ga.list_s = a.list_s;
+    ga.seg_cnt = a.seg_cnt;
+    ga.seg_mall = a.seg_mall;
+    ga.records = records;
+    e = launch_gather_pv(ga, s);
+    g_launches += 1;
+    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+
+    CombineArgs ca{};
+    ca.g = g;
+    ca.mode = kCombineParts;
+    ca.parts = ga.parts;
+    ca.fallback = 1;
+    ca.q = q;
+    ca.k = k;
+    ca.v = v;
+    ca.records = records;
+    ca.out = out;
+    ca.sel_cnt = sel_cnt;
+    g_launches += 1;
+    return cuda_status(launch_combine(ca, s));
+}
+
+int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const void* v,
+                      float* out, void* ws, size_t ws_bytes, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (g.hv > 2 * g.hk) return SAGA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !out || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(out, 4))
+        return SAGA_ERR_INVALID_ARG;
+    if ((st = check_ws(g, ws, ws_bytes))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsLayout L = workspace_layout(g);
+
+    int stages = 4;
+    while (stages > 2 && dense_smem_bytes(g, stages) > static_cast<size_t>(dev.max_smem)) --stages;
+    if (dense_smem_bytes(g, stages) > static_cast<size_t>(dev.max_smem)) return SAGA_ERR_UNSUPPORTED;
+
+    CUtensorMap kmap, vmap;
+    if ((st = encode_cache_map(&kmap, k, g, g.hk, true))) return st;
+    if ((st = encode_cache_map(&vmap, v, g, g.hv, false))) return st;
+    DenseArgs a{};
+    a.g = g;
+    a.C = stream_ctas(g, dev);
+    a.stages = stages;
+    a.q = q;
+    a.records = ws_at<float>(ws, L.records);
+    a.err = ws_at<uint32_t>(ws, L.err);
+    ev_start(s);
+    cudaError_t e = launch_dense(kmap, vmap, a, s);
+    ev_stop(s);
+    g_launches += 1;
+    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+
+    CombineArgs ca{};
+    ca.g = g;
+    ca.mode = kCombineSlots;
+    ca.C = a.C;
+    ca.recs_per_slot = g.WPK;
+    ca.records = a.records;
+    ca.out = out;
+    g_launches += 1;
+    return cuda_status(launch_combine(ca, s));
+}
+
+int saga_workspace_reset(void* ws, size_t ws_bytes, saga_stream_t stream) {
+    if (!ws) return SAGA_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int saga_workspace_error(void* ws, size_t ws_bytes, saga_stream_t stream) {
+    if (!ws || ws_bytes < 256) return SAGA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SAGA_ERR_CUDA;
+    if (cudaMemcpy(&word, ws, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SAGA_ERR_CUDA;
+    if (word && cudaMemset(ws, 0, sizeof word) != cudaSuccess) return SAGA_ERR_CUDA;
+    return (word & kErrTimeout) ? SAGA_ERR_TIMEOUT : SAGA_OK;
+}
+
+const char* saga_status_string(int status) {
+    switch (status) {
+        case SAGA_OK: return "ok";
+        case SAGA_ERR_INVALID_ARG: return "invalid argument";
+        case SAGA_ERR_UNSUPPORTED: return "unsupported shape";
+        case SAGA_ERR_WORKSPACE: return "workspace too small";
+        case SAGA_ERR_CUDA: return "CUDA error";
+        case SAGA_ERR_DEVICE: return "no sm_100 device";
+        case SAGA_ERR_TIMEOUT: return "a bounded device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+uint64_t saga_launch_count(void) { return g_launches.load(); }
+
+void saga_set_kernel_events(void* start_event, void* stop_event) {
+    t_ev_start = static_cast<cudaEvent_t>(start_event);
+    t_ev_stop = static_cast<cudaEvent_t>(stop_event);
+}
+
+int saga_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,121 @@
+// Host-side launch interface of the kernels (internal to libsaga.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "saga_params.h"
+
+namespace saga {
+
+// Streaming query-key kernel over the K cache (TMA pipeline + mma).
+enum StreamMode : int {
+    kStreamLogits = 0,  // write s = q.k/sqrt(d) to logits [b,hq,l]
+    kStreamSelect = 1,  // compare s >= tau and append kept (pos, s) to lists
+};
+
+struct StreamArgs {
+    Geometry g;
+    int C;       // grid size (CTAs), <= kMaxCtas and <= b * tiles
+    int stages;  // pipeline depth
+    const void* q;
+    const float* thresh;
+    float* logits;
+    int32_t* list_idx;
+    float* list_s;
+    int32_t* seg_cnt;
+    float* seg_mall;
+    uint32_t* err;
+};
+
+size_t stream_smem_bytes(int stages);
+cudaError_t launch_qk_stream(int mode, const CUtensorMap& kmap, const StreamArgs& a,
+                             cudaStream_t stream);
+
+// Radix select of the N-th largest logit per row.
+struct RadixArgs {
+    const float* logits;  // [rows][l]
+    long long rows;
+    int l;
+    int N;
+    int chunks;  // CTAs per row
+    uint32_t* hist;
+    uint32_t* state;
+    uint32_t* tickets;
+    float* thresh;
+    uint32_t* err;
+};
+cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream);
+cudaError_t launch_fill(float* p, long long n, float value, cudaStream_t stream);
+
+// Compare + ordered compaction of one logits row per CTA.
+struct SelectArgs {
+    const float* logits;  // [rows][l]
+    const float* thresh;  // [rows]
+    long long rows;
+    int l;
+    int32_t* idx;  // [rows][l]  kept positions, ascending
+    int32_t* cnt;  // [rows]
+};
+cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream);
+
+// Gathered softmax-PV over kept lists -> partial records.
+enum ListMode : int {
+    kListContiguous = 0,  // idx [rows][l], cnt [rows], s from logits
+    kListSegments = 1,    // per (slot, sub-warp) lists from the fused kernel
+};
+struct GatherArgs {
+    Geometry g;
+    int mode;
+    int parts;      // CTAs per row (each takes an equal share of the row's entries)
+    int C;          // kListSegments: grid of the fused kernel
+    int max_lists;  // lists per row at most (kListSegments: slots * WPK; else 1)
+    const void* v;
+    const float* logits;
+    const int32_t* idx;
+    const int32_t* cnt;
+    const int32_t* list_idx;
+    const float* list_s;
+    const int32_t* seg_cnt;
+    const float* seg_mall;
+    float* records;
+};
+size_t gather_smem_bytes(int max_lists);
+cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream);
+
+// Dense flash-decoding kernel (K and V streamed) -> partial records.
+struct DenseArgs {
+    Geometry g;
+    int C;
+    int stages;
+    const void* q;
+    float* records;
+    uint32_t* err;
+};
+size_t dense_stage_bytes(const Geometry& g);
+size_t dense_smem_bytes(const Geometry& g, int stages);
+cudaError_t launch_dense(const CUtensorMap& kmap, const CUtensorMap& vmap, const DenseArgs& a,
+                         cudaStream_t stream);
+
+// Log-sum-exp merge of partial records, plus the empty-set fallback.
+enum CombineMode : int {
+    kCombineParts = 0,     // `parts` records per row (gathered contiguous lists)
+    kCombineSlots = 1,     // slots_of_batch records per row (fused / dense kernels)
+};
+struct CombineArgs {
+    Geometry g;
+    int mode;
+    int parts;
+    int C;
+    int recs_per_slot;  // kCombineSlots: 1 (gathered lists) or WPK (dense kernel)
+    int fallback;  // recompute logits from q/K for rows that kept nothing
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* records;
+    float* out;
+    int32_t* sel_cnt;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+}  // namespace saga

@@ -1,0 +1,129 @@
+"""The C-ABI library: it loads, exports every symbol include/saga.h declares,
+and rejects bad arguments on the host before any CUDA call (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from sparse_decode_attention_saga_b200 import _lib
+from sparse_decode_attention_saga_b200 import build as saga_build
+from sparse_decode_attention_saga_b200.workload import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "saga.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIBRARY):
+        saga_build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(saga_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
+                     "saga_workspace_bytes", "saga_status_string"):
+        assert required in names
+    assert set(names) == set(_lib.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert _lib.status_string(code) not in ("", "unknown status")
+    assert _lib.status_string(-99) == "unknown status"
+
+
+def _ws(n=1 << 16):
+    return torch.zeros(n, dtype=torch.uint8)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(batch=0), _lib.SAGA_ERR_INVALID_ARG),
+    (dict(l_kv=0), _lib.SAGA_ERR_INVALID_ARG),
+    (dict(l_kv=100, l_cap=99), _lib.SAGA_ERR_INVALID_ARG),
+    (dict(head_dim=96), _lib.SAGA_ERR_UNSUPPORTED),
+    (dict(h_k=3, h_q=6), _lib.SAGA_ERR_UNSUPPORTED),
+    (dict(h_q=6, h_k=4), _lib.SAGA_ERR_UNSUPPORTED),
+    (dict(h_q=8, h_v=3), _lib.SAGA_ERR_UNSUPPORTED),
+    (dict(h_q=64, h_k=2, h_v=2), _lib.SAGA_ERR_UNSUPPORTED),  # 32 query heads per key head
+])
+def test_shape_validation(lib, bad, code):
+    base = dict(batch=1, h_q=4, h_k=1, h_v=2, head_dim=64, l_kv=64, l_cap=None)
+    base.update(bad)
+    d = _lib.dims(base["batch"], base["h_q"], base["h_k"], base["h_v"], base["head_dim"],
+                  base["l_kv"], base["l_cap"])
+    assert _lib.workspace_bytes(d, 8) == 0
+    ws = _ws()
+    st = lib.saga_atopn_decode(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, None,
+                               ws.data_ptr(), ws.numel(), None)
+    assert st == code
+
+
+def test_pointer_and_workspace_validation(lib):
+    d = _lib.dims(1, 4, 1, 2, 64, 64)
+    need = _lib.workspace_bytes(d, 8)
+    assert need > 0
+    big = _ws(need + 512)
+    base = (big.data_ptr() + 255) // 256 * 256
+    # null value cache
+    assert lib.saga_atopn_decode(ctypes.byref(d), 16, 16, None, 16, None, 16, None, None,
+                                 base, need, None) == _lib.SAGA_ERR_INVALID_ARG
+    # misaligned key cache
+    assert lib.saga_atopn_decode(ctypes.byref(d), 16, 18, 16, 16, None, 16, None, None,
+                                 base, need, None) == _lib.SAGA_ERR_INVALID_ARG
+    # workspace too small / misaligned
+    assert lib.saga_atopn_decode(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, None,
+                                 base, need - 1, None) == _lib.SAGA_ERR_WORKSPACE
+    assert lib.saga_atopn_decode(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, None,
+                                 base + 8, need, None) == _lib.SAGA_ERR_INVALID_ARG
+    # N <= 0
+    assert lib.saga_topn_refresh(ctypes.byref(d), 0, 16, 16, None, None, 16, base, need,
+                                 None) == _lib.SAGA_ERR_INVALID_ARG
+    # dense needs h_v <= 2 h_k
+    d2 = _lib.dims(1, 8, 1, 8, 64, 64)
+    n2 = _lib.workspace_bytes(d2, 8)
+    ws2 = _ws(n2 + 512)
+    b2 = (ws2.data_ptr() + 255) // 256 * 256
+    assert lib.saga_decode_dense(ctypes.byref(d2), 16, 16, 16, 16, b2, n2, None) == \
+        _lib.SAGA_ERR_UNSUPPORTED
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_a_device_reports_no_device(lib):
+    d = _lib.dims(1, 4, 1, 2, 64, 64)
+    need = _lib.workspace_bytes(d, 8)
+    big = _ws(need + 512)
+    base = (big.data_ptr() + 255) // 256 * 256
+    st = lib.saga_atopn_decode(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, None,
+                               base, need, None)
+    assert st in (_lib.SAGA_ERR_DEVICE, _lib.SAGA_ERR_CUDA)
+
+
+def test_workspace_sizes_for_every_workload(lib):
+    for name, w in CONFIGS.items():
+        d = _lib.dims(w.batch, w.h_q, w.h_k, w.h_v, w.head_dim, w.l_kv, w.cap)
+        n = _lib.workspace_bytes(d, w.N)
+        assert 0 < n < 4 << 30, name
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    missing = str(tmp_path / "libsaga.so")
+    try:
+        with pytest.raises(RuntimeError, match="no CPU fallback"):
+            _lib.load(missing)
+    finally:
+        _lib.load(_lib.LIBRARY)
