@@ -129,6 +129,31 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
                       int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
                       saga_stream_t stream);
 
+/* Allocation-free threshold refresh (the paper has no counterpart; this is
+ * a convenience of this library).  Computes exactly what saga_topn_refresh
+ * computes with logits_in != NULL -- thresh_out[b,i] = the N-th largest of
+ * logits_in[b,i,:] (-inf if N >= l_kv) -- but takes no workspace, for callers
+ * that cannot allocate device memory on the decode path (a plugin inside a
+ * host engine that owns all device memory and gives its plugins no
+ * allocator; a loop that must not call cudaMalloc after start-up because it
+ * can synchronise the device or fail under memory pressure).  Only head_dim-
+ * independent fields of dims are used (batch, h_q, l_kv).
+ *   - Scratch: a 16 MiB file-scope device array inside libsaga.so, held by
+ *     every GPU that loads the library until the process exits; it covers
+ *     batch*h_q <= 682 rows.  More rows return SAGA_ERR_WORKSPACE and
+ *     enqueue nothing.  Nothing is allocated: no cudaMalloc/cudaFree, no
+ *     allocating library call.
+ *   - First call per device: looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call clears the array's histograms on `stream` and then reuses
+ *     it, so calls whose work overlaps on the GPU (other streams, other host
+ *     threads) race on the shared scratch: order them on one stream.
+ * Errors: SAGA_ERR_INVALID_ARG (null/misaligned pointer, N <= 0, bad dims),
+ * SAGA_ERR_WORKSPACE (too many rows), SAGA_ERR_DEVICE, SAGA_ERR_CUDA. */
+int saga_topn_refresh_noalloc(const saga_dims* dims, int32_t N, const float* logits_in,
+                              float* thresh_out, saga_stream_t stream);
+
 /* Enqueue a zeroing of the workspace (sticky flags included). */
 int saga_workspace_reset(void* ws, size_t ws_bytes, saga_stream_t stream);
 

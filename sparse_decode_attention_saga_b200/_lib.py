@@ -26,7 +26,7 @@ SAGA_ERR_TIMEOUT = -6
 EXPORTS = (
     "saga_workspace_bytes", "saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
     "saga_workspace_reset", "saga_workspace_error", "saga_status_string", "saga_launch_count",
-    "saga_set_kernel_events", "saga_version",
+    "saga_set_kernel_events", "saga_version", "saga_topn_refresh_noalloc",
 )
 
 
@@ -64,6 +64,8 @@ def load(path: str | None = None):
         lib.saga_decode_dense.argtypes = [D, P, P, P, P, P, SZ, P]
         lib.saga_topn_refresh.argtypes = [D, I32, P, P, P, P, P, P, SZ, P]
         lib.saga_atopn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.saga_topn_refresh_noalloc.argtypes = [D, I32, P, P, P]
+        lib.saga_topn_refresh_noalloc.restype = ctypes.c_int
         lib.saga_workspace_reset.argtypes = [P, SZ, P]
         lib.saga_workspace_error.argtypes = [P, SZ, P]
         lib.saga_status_string.argtypes = [ctypes.c_int]
@@ -129,6 +131,14 @@ def atopn_decode(d, q, k, v, thresh, logits_in, out, sel_idx, sel_cnt, ws, strea
                                   _ptr(logits_in), _ptr(out), _ptr(sel_idx), _ptr(sel_cnt),
                                   _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
     _check("saga_atopn_decode", st)
+
+
+def topn_refresh_noalloc(d, N, logits_in, thresh_out, stream=None) -> None:
+    """Threshold refresh without a workspace (scratch is a fixed array inside
+    the library); for callers that cannot allocate device memory."""
+    st = load().saga_topn_refresh_noalloc(ctypes.byref(d), int(N), _ptr(logits_in),
+                                          _ptr(thresh_out), _stream(stream))
+    _check("saga_topn_refresh_noalloc", st)
 
 
 def workspace_reset(ws, stream=None) -> None:

@@ -46,6 +46,8 @@ struct RadixArgs {
     uint32_t* err;
 };
 cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream);
+// Adds n to the library's launch counter (saga_launch_count).
+void note_launches(int n);
 cudaError_t launch_fill(float* p, long long n, float value, cudaStream_t stream);
 
 // Compare + ordered compaction of one logits row per CTA.
