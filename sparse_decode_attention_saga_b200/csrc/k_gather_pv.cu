@@ -6,19 +6,21 @@
 // value rows of kept positions, from value head vh(i) = i*h_v/h_q (SAGA,
 // Key Contributions #3).
 //
-// A row's kept entries live in one or more ascending lists: one contiguous
-// list from the compare/compact kernel (kListContiguous), or one list per
+// A row's kept entries live in one or more ascending lists of (position,
+// logit) pairs: one contiguous list from the compare/compact kernel
+// (kListContiguous), or one list per
 // (streaming CTA slot, consumer warp) from the fused kernel (kListSegments).
 // Grid (parts, rows): every CTA builds the row's list table (counts and
 // exclusive prefix) in shared memory and takes an equal share of the row's
 // flattened entries, so the work is balanced whatever the lists' lengths.
-// The share is processed in batches: the batch's (position, logit) pairs are
-// copied to shared memory with coalesced loads, its largest logit updates
-// the running max (online rescaling between batches), and then every lane
-// group gathers value rows with 16-byte loads, many rows in flight per lane,
-// weights them by exp(s - m) and accumulates in fp32.  The share's (m, sum of
-// weights, count, row max, unnormalised output) goes to a partial record
-// that the combine kernel merges.
+// Each warp then works through its own contiguous part of that share without
+// block barriers: 32 entries at a time, one (position, logit) per lane read
+// with coalesced loads one round ahead, and 16-byte value-row loads by lane
+// groups (8 or 16 lanes per row), weighted by exp(s - m) and accumulated in
+// fp32.  m is the row's largest logit, which is always kept when anything is
+// (tau_eff <= max), so no running max is needed.  The share's (m, sum of
+// weights, count, row max, unnormalised output) record is merged across
+// shares by the combine kernel.
 #include "saga_device.cuh"
 #include "saga_kernels.h"
 
@@ -28,18 +30,25 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBatch = 2048;  // entries staged in shared memory at a time
+#ifndef SAGA_GATHER_INFLIGHT
+#define SAGA_GATHER_INFLIGHT 4
+#endif
+#ifndef SAGA_GATHER_MINBLOCKS
+#define SAGA_GATHER_MINBLOCKS 4
+#endif
+// value-row loads in flight per lane group, and CTAs per SM the register
+// budget is sized for (tuning constants)
+constexpr int kGatherInflight = SAGA_GATHER_INFLIGHT;
+constexpr int kGatherMinBlocks = SAGA_GATHER_MINBLOCKS;
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 3) gather_pv_kernel(const GatherArgs a) {
+__global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(const GatherArgs a) {
     constexpr int LPR = D * 2 / 16;    // lanes per value row (16 B each)
     constexpr int RPI = 32 / LPR;      // value rows per warp instruction
     constexpr int UNROLL = 8;
     constexpr int MBW = 128 / D;
 
     extern __shared__ int table[];     // pre[max_lists + 1], start[max_lists]
-    __shared__ int ent_pos[kBatch];
-    __shared__ float ent_s[kBatch];
     __shared__ float red_m[kWarps];
     __shared__ float red_l[kWarps];
     __shared__ float red_o[kWarps][D];
@@ -66,6 +75,7 @@ __global__ void __launch_bounds__(kThreads, 3) gather_pv_kernel(const GatherArgs
             start[0] = 0;
             row_base = row * g.l;
         }
+        m_all = __ldg(a.rowmax + row);
         __syncthreads();
     } else {
         const long long T = static_cast<long long>(g.b) * g.tiles;
@@ -126,74 +136,67 @@ __global__ void __launch_bounds__(kThreads, 3) gather_pv_kernel(const GatherArgs
     const int e0 = static_cast<int>(static_cast<long long>(total) * part / a.parts);
     const int e1 = static_cast<int>(static_cast<long long>(total) * (part + 1) / a.parts);
     const int n = e1 - e0;
+    // each warp owns a contiguous sub-share and needs no block barrier
+    const int w0 = e0 + static_cast<int>(static_cast<long long>(n) * warp / kWarps);
+    const int w1 = e0 + static_cast<int>(static_cast<long long>(n) * (warp + 1) / kWarps);
+    // Softmax reference: whenever a row keeps anything its largest kept logit
+    // is the row's largest logit (tau_eff <= max), so exp(s - m) needs no
+    // running max and no rescaling.
+    const float m = m_all;
 
     const int grp = lane / LPR, col0 = (lane % LPR) * 8;
     float acc[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] = 0.f;
     float lsum = 0.f;
-    float m = -kInf;
     const __nv_bfloat16* vbase = reinterpret_cast<const __nv_bfloat16*>(a.v) +
                                  (static_cast<size_t>(bb) * g.l_cap * g.hv + vh) * D + col0;
     const size_t vstride = static_cast<size_t>(g.hv) * D;
-    constexpr int step = kWarps * RPI;
+    constexpr int ROUNDS = 32 / RPI;   // value-row loads per lane per 32 entries
+    constexpr int INFLIGHT = ROUNDS < kGatherInflight ? ROUNDS : kGatherInflight;
 
-    // first list that holds entry e0
-    int jl = 0;
-    while (jl + 1 < nl && pre[jl + 1] <= e0) ++jl;
-
-    for (int b0 = e0; b0 < e1; b0 += kBatch) {
-        const int b1 = min(e1, b0 + kBatch);
-        // ---- stage the batch's (position, logit) pairs, list by list
-        float mloc = -kInf;
-        for (int j = jl; j < nl && pre[j] < b1; ++j) {
-            const int lo = max(b0, pre[j]), hi = min(b1, pre[j + 1]);
-            const long long src = row_base + start[j] - pre[j];
-            for (int e = lo + tid; e < hi; e += kThreads) {
-                int pos;
-                float s;
-                if (a.mode == kListContiguous) {
-                    pos = __ldg(a.idx + src + e);
-                    s = __ldg(a.logits + row * g.l + pos);
-                } else {
-                    pos = __ldg(a.list_idx + src + e);
-                    s = __ldg(a.list_s + src + e);
-                }
-                ent_pos[e - b0] = pos;
-                ent_s[e - b0] = s;
-                mloc = fmaxf(mloc, s);
+    // entry e -> (position, logit); out-of-range entries give (0, -inf)
+    auto fetch = [&](int e, int& pos, float& s) {
+        pos = 0;
+        s = -kInf;
+        if (e < w1) {
+            int lo = 0, hi = nl - 1;  // last list j with pre[j] <= e
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (pre[mid] <= e) lo = mid; else hi = mid - 1;
             }
+            const long long at = row_base + start[lo] + (e - pre[lo]);
+            pos = __ldg((a.mode == kListContiguous ? a.idx : a.list_idx) + at);
+            s = __ldg(a.list_s + at);
         }
-        while (jl + 1 < nl && pre[jl + 1] <= b1) ++jl;
-        mloc = warp_max(mloc);
-        if (lane == 0) red_m[warp] = mloc;
-        __syncthreads();
-        float m_new = m;
+    };
+    int nxt_pos;
+    float nxt_s;
+    fetch(w0 + lane, nxt_pos, nxt_s);
+    for (int base = w0; base < w1; base += 32) {
+        // one entry per lane; the next round's entries are already in flight
+        const int pos = nxt_pos;
+        const float s = nxt_s;
+        fetch(base + 32 + lane, nxt_pos, nxt_s);
+        const float p_lane = base + lane < w1 ? __expf(s - m) : 0.f;
+        lsum += p_lane;
+        // lane group grp gathers entries grp, grp+RPI, ... of the 32
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) m_new = fmaxf(m_new, red_m[w]);
-        const float alpha = m > -kInf ? __expf(m - m_new) : 0.f;
-        lsum *= alpha;
+        for (int r0 = 0; r0 < ROUNDS; r0 += INFLIGHT) {
+            uint4 raw[INFLIGHT];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) acc[c] *= alpha;
-        m = m_new;
-
-        // ---- gather the batch's value rows
-        const int nb = b1 - b0;
-        for (int e = warp * RPI + grp; e < nb; e += step * UNROLL) {
-            uint4 raw[UNROLL];
-            float p[UNROLL];
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const int eu = e + u * step;
-                const bool ok = eu < nb;
-                const int pos = ok ? ent_pos[eu] : 0;
-                p[u] = ok ? __expf(ent_s[eu] - m) : 0.f;
-                raw[u] = ok ? __ldg(reinterpret_cast<const uint4*>(vbase + pos * vstride))
-                            : make_uint4(0u, 0u, 0u, 0u);
+            for (int u = 0; u < INFLIGHT; ++u) {
+                const int k = (r0 + u) * RPI + grp;
+                const int pk = __shfl_sync(0xffffffffu, pos, k);
+                raw[u] = base + k < w1 ? __ldg(reinterpret_cast<const uint4*>(vbase + pk * vstride))
+                                       : make_uint4(0u, 0u, 0u, 0u);
             }
+            float p[INFLIGHT];
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                lsum += p[u];
+            for (int u = 0; u < INFLIGHT; ++u)
+                p[u] = __shfl_sync(0xffffffffu, p_lane, (r0 + u) * RPI + grp);
+#pragma unroll
+            for (int u = 0; u < INFLIGHT; ++u) {
                 const uint32_t w4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -202,11 +205,10 @@ __global__ void __launch_bounds__(kThreads, 3) gather_pv_kernel(const GatherArgs
                 }
             }
         }
-        __syncthreads();  // the next batch overwrites the staged entries
     }
 
-    // every lane of a row group saw each of the group's weights: count once
-    lsum = (lane % LPR == 0) ? lsum : 0.f;
+    // reduce the row groups of the warp (lanes with equal col0), then merge the
+    // warps' (max, sum, output) with log-sum-exp weights
 #pragma unroll
     for (int o = LPR; o < 32; o <<= 1) {
 #pragma unroll
@@ -219,7 +221,6 @@ __global__ void __launch_bounds__(kThreads, 3) gather_pv_kernel(const GatherArgs
     }
     if (lane == 0) red_l[warp] = lsum;
     __syncthreads();
-
     float* rec = a.records + (static_cast<size_t>(row) * g.S_cap * g.WPK + part) * g.rec;
     for (int c = tid; c < D; c += kThreads) {
         float o = 0.f;
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 3) gather_pv_kernel(const GatherArgs
         rec[0] = n > 0 ? m : -kInf;
         rec[1] = l;
         rec[2] = __int_as_float(n);
-        rec[3] = a.mode == kListContiguous ? (n > 0 ? m : -kInf) : m_all;
+        rec[3] = m_all;
     }
 }
 

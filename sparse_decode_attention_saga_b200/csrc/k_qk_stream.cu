@@ -28,7 +28,7 @@ namespace {
 
 
 template <int D, int NT, int MODE>
-__global__ void __launch_bounds__(kStreamThreads, 1)
+__global__ void __launch_bounds__(kStreamThreads, 2)
     qk_stream_kernel(const __grid_constant__ CUtensorMap kmap, const StreamArgs a) {
     constexpr int MBW = 128 / D;
     constexpr int DH = D / 64;
@@ -63,12 +63,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         if (lane == 0) {
             prefetch_tensor_map(&kmap);
             int issued = 0;
+            int bb = static_cast<int>(t0 / g.tiles);
+            int tl = static_cast<int>(t0 - static_cast<long long>(bb) * g.tiles);
+            int st = 0;
+            uint32_t phase = 0;
             for (int k = 0; k < ntile; ++k) {
-                const int st = k % stages;
-                if (!mbar_wait(&empty[st], ((k / stages) & 1) ^ 1, abort_flag)) break;
-                const long long t = t0 + k;
-                const int bb = static_cast<int>(t / g.tiles);
-                const int tl = static_cast<int>(t - static_cast<long long>(bb) * g.tiles);
+                if (!mbar_wait(&empty[st], phase ^ 1, abort_flag)) break;
                 const int z = bb * g.l_cap + tl * g.P;
                 mbar_arrive_expect_tx(&full[st], kStageBytes);
                 uint8_t* dst = smem + static_cast<size_t>(st) * kStageBytes;
@@ -77,6 +77,14 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                         tma_load_3d(dst + (kh * DH + dh) * g.P * 128, &kmap, &full[st], dh * 64,
                                     kh, z);
                 issued = k + 1;
+                if (++tl == g.tiles) {
+                    tl = 0;
+                    ++bb;
+                }
+                if (++st == stages) {
+                    st = 0;
+                    phase ^= 1;
+                }
             }
             // Drain: the last load armed on each stage must land before exit.
             int dummy = 0;
@@ -141,17 +149,17 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     };
 
     bool ok = true;
+    int bb = static_cast<int>(t0 / g.tiles);
+    int tl = static_cast<int>(t0 - static_cast<long long>(bb) * g.tiles);
+    int st = 0;
+    uint32_t phase = 0;
     for (int k = 0; k < ntile; ++k) {
-        const long long t = t0 + k;
-        const int bb = static_cast<int>(t / g.tiles);
-        const int tl = static_cast<int>(t - static_cast<long long>(bb) * g.tiles);
         if (bb != cur_bb) {
             if (cur_bb >= 0) end_segment(cur_bb);
             begin_segment(bb);
             cur_bb = bb;
         }
-        const int st = k % stages;
-        const bool got = mbar_wait(&full[st], (k / stages) & 1, abort_flag);
+        const bool got = mbar_wait(&full[st], phase, abort_flag);
         if (!__all_sync(0xffffffffu, got)) {
             ok = false;
             break;
@@ -160,6 +168,10 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         qk_mma<D, NT, MBW>(stage0 + st * kStageBytes, g.P, kh, mb0, qf, acc, lane);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);
+        if (++st == stages) {
+            st = 0;
+            phase ^= 1;
+        }
 
         const int pos0 = tl * g.P + mb0 * 16 + gq;
 #pragma unroll
@@ -194,6 +206,10 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                         }
                     }
             }
+        if (++tl == g.tiles) {
+            tl = 0;
+            ++bb;
+        }
     }
     if (cur_bb >= 0) end_segment(cur_bb);
     if (!ok && lane == 0) raise_device_error(a.err, kErrTimeout);

@@ -8,8 +8,8 @@
 // exact and needs no sort.
 //
 // Pass p, grid (chunks, rows): each CTA histograms the digit of the keys of
-// its chunk that match the prefix fixed by the earlier passes (warp-
-// aggregated shared atomics), adds its histogram to the row's global one,
+// its chunk that match the prefix fixed by the earlier passes (shared-memory
+// atomics), adds its histogram to the row's global one,
 // and takes a ticket; the CTA that takes the last ticket scans the histogram
 // from the top bin, fixes the digit that holds the rank, and stores
 // (prefix, rank) for the next pass, or the threshold after the last pass.
@@ -47,8 +47,9 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t& e
     return total;
 }
 
-template <int PASS>
+template <int PASS, int VEC>
 __global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a) {
+    constexpr int kLoadsV = kLoads / VEC;  // VEC-wide loads per thread per round
     constexpr int shift = PASS == 0 ? 21 : (PASS == 1 ? 10 : 0);
     constexpr int width = PASS == 2 ? 10 : 11;
     constexpr int nb = 1 << width;
@@ -59,7 +60,7 @@ __global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a)
     __shared__ uint32_t warp_tot[kThreads / 32];
     __shared__ int is_last;
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const long long row = blockIdx.y;
     const int chunk = blockIdx.x;
     for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
@@ -67,31 +68,35 @@ __global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a)
     __syncthreads();
 
     const float* src = a.logits + row * a.l;
-    const int per = (a.l + a.chunks - 1) / a.chunks;
+    const int per = ((a.l + a.chunks - 1) / a.chunks + 3) & ~3;  // multiple of 4
     const int j0 = chunk * per;
     const int j1 = min(a.l, j0 + per);
-    // kLoads independent coalesced loads per thread per round keep enough
-    // bytes in flight to stream the logits at HBM speed.
-    for (int base = j0; base < j1; base += kLoads * kThreads) {
-        float v[kLoads];
+    // 64 bytes of independent coalesced loads per thread per round (16-byte
+    // loads when the rows are 16-byte aligned) keep enough bytes in flight to
+    // stream the logits at HBM speed.
+    for (int base = j0; base < j1; base += kLoadsV * kThreads * VEC) {
+        float v[kLoadsV][VEC];
 #pragma unroll
-        for (int k = 0; k < kLoads; ++k) {
-            const int j = base + k * kThreads + tid;
-            v[k] = j < j1 ? __ldg(src + j) : 0.f;
+        for (int k = 0; k < kLoadsV; ++k) {
+            const int j = base + (k * kThreads + tid) * VEC;
+            if (VEC == 4 && j + VEC <= j1) {
+                const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
+                const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int c = 0; c < VEC; ++c) v[k][c] = xs[c];
+            } else {
+#pragma unroll
+                for (int c = 0; c < VEC; ++c) v[k][c] = j + c < j1 ? __ldg(src + j + c) : 0.f;
+            }
         }
 #pragma unroll
-        for (int k = 0; k < kLoads; ++k) {
-            const int j = base + k * kThreads + tid;
-            const bool valid = j < j1;
-            const uint32_t key = float_to_key(v[k]);
-            const bool cand = valid && (PASS == 0 || (key >> high) == prefix);
-            const uint32_t digit = (key >> shift) & (nb - 1);
-            if (PASS == 0) {
-                // most keys are candidates: aggregate equal digits across the warp
-                const uint32_t peers = __match_any_sync(0xffffffffu, cand ? digit : 0xffffffffu);
-                if (cand && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
-            } else if (cand) {
-                atomicAdd(&hist[digit], 1u);
+        for (int k = 0; k < kLoadsV; ++k) {
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) {
+                const int j = base + (k * kThreads + tid) * VEC + c;
+                const uint32_t key = float_to_key(v[k][c]);
+                const bool cand = j < j1 && (PASS == 0 || (key >> high) == prefix);
+                if (cand) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
             }
         }
     }
@@ -152,9 +157,16 @@ __global__ void fill_kernel(float* p, long long n, float value) {
 
 cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream) {
     const dim3 grid(a.chunks, static_cast<unsigned>(a.rows));
-    radix_pass_kernel<0><<<grid, kThreads, 0, stream>>>(a);
-    radix_pass_kernel<1><<<grid, kThreads, 0, stream>>>(a);
-    radix_pass_kernel<2><<<grid, kThreads, 0, stream>>>(a);
+    const bool vec = (a.l % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.logits) & 15u) == 0);
+    if (vec) {
+        radix_pass_kernel<0, 4><<<grid, kThreads, 0, stream>>>(a);
+        radix_pass_kernel<1, 4><<<grid, kThreads, 0, stream>>>(a);
+        radix_pass_kernel<2, 4><<<grid, kThreads, 0, stream>>>(a);
+    } else {
+        radix_pass_kernel<0, 1><<<grid, kThreads, 0, stream>>>(a);
+        radix_pass_kernel<1, 1><<<grid, kThreads, 0, stream>>>(a);
+        radix_pass_kernel<2, 1><<<grid, kThreads, 0, stream>>>(a);
+    }
     return cudaGetLastError();
 }
 

@@ -7,11 +7,15 @@
 // are silent): tau_eff = min(tau, row max), i.e. when a stale threshold lies
 // above every logit the row's maximal entries are kept.
 //
-// One CTA per (batch, query head) row.  Each round covers 16 x 256 positions:
-// every warp ballots its 32 positions per sub-round, the 128 warp counts are
-// prefix-summed by warp 0, and each kept lane writes its position at the
-// scanned offset, so the output is ascending.  If nothing passed (only
-// possible when tau > row max) the row is compacted again against its max.
+// One CTA of 256 threads per (batch, query head) row.  A round covers
+// 4 x 256 x VEC positions: each thread reads VEC consecutive logits per
+// sub-round (16-byte loads when rows are 16-byte aligned), counts its kept
+// ones, the counts are prefix-summed inside the warp (shuffles) and across
+// the 8 warps x 4 sub-rounds (warp 0), and every kept position (and its
+// logit, for the gather kernel) is written at its rank, so the output is
+// ascending.  The row's largest logit is stored for the gather kernel's
+// softmax.  If nothing passed (only possible when tau > row max) the row is
+// compacted again against its max.
 #include "saga_device.cuh"
 #include "saga_kernels.h"
 
@@ -21,83 +25,106 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSub = 16;                    // sub-rounds per round
-constexpr int kRound = kSub * kThreads;     // positions per round
+constexpr int kSub = 4;  // sub-rounds per round; kSub * kWarps == 32 counts per round
 
+template <int VEC>
 __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectArgs a) {
+    constexpr int kRound = kSub * kThreads * VEC;  // positions per round
     __shared__ int counts[kSub * kWarps];
     __shared__ int offsets[kSub * kWarps];
     __shared__ int round_total;
-    __shared__ float warp_max_s[kWarps];
+    __shared__ float red[kWarps];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long row = blockIdx.x;
     const float* src = a.logits + row * a.l;
     int32_t* dst = a.idx + row * a.l;
+    float* sdst = a.s + row * a.l;
     const float tau = __ldg(a.thresh + row);
-    constexpr float kNegInf = -kInf;
 
-    float tmax = kNegInf;
+    float tmax = -kInf;
     int total = 0;
     for (int pass = 0; pass < 2; ++pass) {
         float t_eff = tau;
-        if (pass == 1) {
-            // Only reached when nothing was kept: keep the row's maximum.
-            tmax = warp_max(tmax);
-            if (lane == 0) warp_max_s[warp] = tmax;
-            __syncthreads();
-            float m = warp_max_s[0];
-            for (int w = 1; w < kWarps; ++w) m = fmaxf(m, warp_max_s[w]);
-            t_eff = m;
-        }
+        if (pass == 1) t_eff = red[0];  // only reached when nothing was kept: keep the max
         total = 0;
         for (int base = 0; base < a.l; base += kRound) {
-            float v[kSub];
+            float v[kSub][VEC];
 #pragma unroll
             for (int k = 0; k < kSub; ++k) {
-                const int j = base + k * kThreads + tid;
-                v[k] = j < a.l ? __ldg(src + j) : kNegInf;
+                const int j = base + (k * kThreads + tid) * VEC;
+                if (VEC == 4 && j + VEC <= a.l) {
+                    const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
+                    const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int c = 0; c < VEC; ++c) v[k][c] = xs[c];
+                } else {
+#pragma unroll
+                    for (int c = 0; c < VEC; ++c) v[k][c] = j + c < a.l ? __ldg(src + j + c) : -kInf;
+                }
             }
-            uint32_t ball[kSub];
+            uint32_t kb[kSub];
+            int lane_off[kSub];
 #pragma unroll
             for (int k = 0; k < kSub; ++k) {
-                const int j = base + k * kThreads + tid;
-                if (pass == 0) tmax = fmaxf(tmax, v[k]);
-                ball[k] = __ballot_sync(0xffffffffu, j < a.l && v[k] >= t_eff);
-                if (lane == 0) counts[k * kWarps + warp] = __popc(ball[k]);
+                const int j = base + (k * kThreads + tid) * VEC;
+                kb[k] = 0u;
+#pragma unroll
+                for (int c = 0; c < VEC; ++c) {
+                    if (pass == 0) tmax = fmaxf(tmax, v[k][c]);
+                    if (j + c < a.l && v[k][c] >= t_eff) kb[k] |= 1u << c;
+                }
+                const int mine = __popc(kb[k]);
+                int inc = mine;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int x = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += x;
+                }
+                lane_off[k] = inc - mine;
+                if (lane == 31) counts[k * kWarps + warp] = inc;
             }
             __syncthreads();
             if (warp == 0) {
-                // exclusive scan of the 128 counts in position order (k major, warp minor)
-                int c[4], s = 0;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    c[u] = counts[lane * 4 + u];
-                    s += c[u];
-                }
-                int inc = s;
+                // exclusive scan of the 32 counts in position order (k major, warp minor)
+                const int c = counts[lane];
+                int inc = c;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    const int n = __shfl_up_sync(0xffffffffu, inc, o);
-                    if (lane >= o) inc += n;
+                    const int x = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += x;
                 }
-                int run = inc - s;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    offsets[lane * 4 + u] = run;
-                    run += c[u];
-                }
+                offsets[lane] = inc - c;
                 if (lane == 31) round_total = inc;
             }
             __syncthreads();
 #pragma unroll
             for (int k = 0; k < kSub; ++k) {
-                if (ball[k] & (1u << lane)) {
-                    const int at = total + offsets[k * kWarps + warp] + __popc(ball[k] & lanemask_lt());
-                    dst[at] = base + k * kThreads + tid;
+                if (!kb[k]) continue;
+                int at = total + offsets[k * kWarps + warp] + lane_off[k];
+                const int j = base + (k * kThreads + tid) * VEC;
+#pragma unroll
+                for (int c = 0; c < VEC; ++c) {
+                    if (kb[k] & (1u << c)) {
+                        dst[at] = j + c;
+                        sdst[at] = v[k][c];
+                        ++at;
+                    }
                 }
             }
             total += round_total;
+            __syncthreads();
+        }
+        if (pass == 0) {
+            tmax = warp_max(tmax);
+            if (lane == 0) red[warp] = tmax;
+            __syncthreads();
+            if (tid == 0) {
+                float m = red[0];
+                for (int w = 1; w < kWarps; ++w) m = fmaxf(m, red[w]);
+                red[0] = m;
+                a.rowmax[row] = m;
+            }
             __syncthreads();
         }
         if (total > 0) break;
@@ -108,7 +135,11 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
 }  // namespace
 
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream) {
-    select_compact_kernel<<<static_cast<unsigned>(a.rows), kThreads, 0, stream>>>(a);
+    const bool vec = (a.l % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.logits) & 15u) == 0);
+    if (vec)
+        select_compact_kernel<4><<<static_cast<unsigned>(a.rows), kThreads, 0, stream>>>(a);
+    else
+        select_compact_kernel<1><<<static_cast<unsigned>(a.rows), kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -21,7 +21,16 @@ using namespace saga;
 
 namespace {
 
-constexpr int kStreamStages = 6;  // 6 x 32 KB of K in flight per SM
+// Pipeline depth and CTAs per SM of the streaming kernels (tuning constants):
+// 3 x 32 KB of K per CTA, two CTAs per SM.
+#ifndef SAGA_STREAM_STAGES
+#define SAGA_STREAM_STAGES 3
+#endif
+#ifndef SAGA_STREAM_CTAS_PER_SM
+#define SAGA_STREAM_CTAS_PER_SM 2
+#endif
+constexpr int kStreamStages = SAGA_STREAM_STAGES;
+constexpr int kStreamCtasPerSm = SAGA_STREAM_CTAS_PER_SM;
 constexpr int kMaxDevices = 64;
 
 std::atomic<uint64_t> g_launches{0};
@@ -138,11 +147,11 @@ int max_slots(const Geometry& g, long long T, int C) {
     return m;
 }
 
-// Grid of the streaming kernels: one CTA per SM, at most one per tile, and
+// Grid of the streaming kernels: `per_sm` CTAs per SM, at most one per tile, and
 // never more partial-record slots per batch row than the workspace holds.
-int stream_ctas(const Geometry& g, const DeviceInfo& dev) {
+int stream_ctas(const Geometry& g, const DeviceInfo& dev, int per_sm = kStreamCtasPerSm) {
     const long long T = static_cast<long long>(g.b) * g.tiles;
-    long long c = dev.sms;
+    long long c = static_cast<long long>(dev.sms) * per_sm;
     if (c > kMaxCtas) c = kMaxCtas;
     if (c > T) c = T;
     int C = static_cast<int>(c < 1 ? 1 : c);
@@ -159,6 +168,31 @@ int gather_parts(const Geometry& g, const DeviceInfo& dev) {
     if (parts > cap) parts = cap;
     return static_cast<int>(parts < 1 ? 1 : parts);
 }
+
+}  // namespace
+
+namespace saga {
+// CTAs per row of the radix passes.  Cost model: waves of 8 CTAs per SM, each
+// wave as long as one CTA's share of the row plus a fixed per-CTA cost (its
+// 2048-bin histogram is cleared and flushed) worth about 3000 logits.
+int radix_chunks(long long rows, int l, int sms) {
+    const long long slots = 8ll * sms;
+    const long long max_chunks = (l + 4095) / 4096;
+    long long best = 1;
+    double best_cost = 1e300;
+    for (long long c = 1; c <= max_chunks && c <= 64; ++c) {
+        const long long waves = (rows * c + slots - 1) / slots;
+        const double cost = static_cast<double>(waves) * (static_cast<double>((l + c - 1) / c) + 3000.0);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = c;
+        }
+    }
+    return static_cast<int>(best);
+}
+}  // namespace saga
+
+namespace {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGA_OK : SAGA_ERR_CUDA; }
 
@@ -241,10 +275,7 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
     r.rows = rows;
     r.l = g.l;
     r.N = N;
-    long long chunks = (8ll * dev.sms + rows - 1) / rows;
-    const long long max_chunks = (g.l + 2047) / 2048;
-    if (chunks > max_chunks) chunks = max_chunks;
-    r.chunks = static_cast<int>(chunks < 1 ? 1 : chunks);
+    r.chunks = radix_chunks(rows, g.l, dev.sms);
     r.hist = ws_at<uint32_t>(ws, L.hist);
     r.state = ws_at<uint32_t>(ws, L.state);
     r.tickets = ws_at<uint32_t>(ws, L.tickets);
@@ -289,7 +320,9 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         sa.rows = rows;
         sa.l = g.l;
         sa.idx = sel_idx ? sel_idx : ws_at<int32_t>(ws, L.list_idx);
+        sa.s = ws_at<float>(ws, L.list_s);
         sa.cnt = ws_at<int32_t>(ws, L.cnt);
+        sa.rowmax = ws_at<float>(ws, L.rowmax);
         cudaError_t e = launch_select_compact(sa, s);
         g_launches += 1;
         if (e != cudaSuccess) return SAGA_ERR_CUDA;
@@ -300,9 +333,10 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         ga.parts = gather_parts(g, dev);
         ga.max_lists = 1;
         ga.v = v;
-        ga.logits = logits;
         ga.idx = sa.idx;
+        ga.list_s = sa.s;
         ga.cnt = sa.cnt;
+        ga.rowmax = sa.rowmax;
         ga.records = records;
         e = launch_gather_pv(ga, s);
         g_launches += 1;
@@ -396,7 +430,7 @@ int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const
     if ((st = encode_cache_map(&vmap, v, g, g.hv, false))) return st;
     DenseArgs a{};
     a.g = g;
-    a.C = stream_ctas(g, dev);
+    a.C = stream_ctas(g, dev, 1);
     a.stages = stages;
     a.q = q;
     a.records = ws_at<float>(ws, L.records);

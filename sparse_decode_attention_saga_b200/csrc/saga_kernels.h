@@ -46,6 +46,8 @@ struct RadixArgs {
     uint32_t* err;
 };
 cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream);
+// CTAs per row for the radix passes (cost model over waves and per-CTA overhead).
+int radix_chunks(long long rows, int l, int sms);
 // Adds n to the library's launch counter (saga_launch_count).
 void note_launches(int n);
 cudaError_t launch_fill(float* p, long long n, float value, cudaStream_t stream);
@@ -57,7 +59,9 @@ struct SelectArgs {
     long long rows;
     int l;
     int32_t* idx;  // [rows][l]  kept positions, ascending
+    float* s;      // [rows][l]  their logits, same order
     int32_t* cnt;  // [rows]
+    float* rowmax; // [rows]     largest logit of the row
 };
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream);
 
@@ -73,11 +77,11 @@ struct GatherArgs {
     int C;          // kListSegments: grid of the fused kernel
     int max_lists;  // lists per row at most (kListSegments: slots * WPK; else 1)
     const void* v;
-    const float* logits;
-    const int32_t* idx;
-    const int32_t* cnt;
-    const int32_t* list_idx;
-    const float* list_s;
+    const int32_t* idx;       // kListContiguous: positions [rows][l]
+    const int32_t* cnt;       // kListContiguous: counts [rows]
+    const float* rowmax;      // kListContiguous: largest logit per row [rows]
+    const int32_t* list_idx;  // kListSegments: positions [rows][l_pad]
+    const float* list_s;      // logits of the listed entries (row stride l or l_pad)
     const int32_t* seg_cnt;
     const float* seg_mall;
     float* records;

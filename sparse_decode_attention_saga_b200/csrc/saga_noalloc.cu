@@ -103,10 +103,7 @@ extern "C" int saga_topn_refresh_noalloc(const saga_dims* dims, int32_t N, const
     r.rows = rows;
     r.l = l;
     r.N = N;
-    long long chunks = (8ll * sms + rows - 1) / rows;
-    const long long max_chunks = (l + 2047) / 2048;
-    if (chunks > max_chunks) chunks = max_chunks;
-    r.chunks = static_cast<int>(chunks < 1 ? 1 : chunks);
+    r.chunks = radix_chunks(rows, l, sms);
     r.hist = hist;
     r.state = state;
     r.tickets = tickets;

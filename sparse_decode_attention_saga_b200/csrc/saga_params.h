@@ -69,6 +69,7 @@ struct WsLayout {
     size_t state;     // uint32 [b*hq][2]  (prefix, rank)
     size_t tickets;   // uint32 [b*hq]
     size_t cnt;       // int32  [b*hq]
+    size_t rowmax;    // float  [b*hq]
     size_t seg_cnt;   // int32  [b*hq][S_cap][WPK]
     size_t seg_mall;  // float  [b*hq][S_cap][WPK]
     size_t list_idx;  // int32  [b*hq][l_pad]
@@ -94,6 +95,7 @@ inline WsLayout workspace_layout(const Geometry& g) {
     w.state = take(rows * 2 * sizeof(uint32_t));
     w.tickets = take(rows * sizeof(uint32_t));
     w.cnt = take(rows * sizeof(int32_t));
+    w.rowmax = take(rows * sizeof(float));
     w.seg_cnt = take(rows * g.S_cap * g.WPK * sizeof(int32_t));
     w.seg_mall = take(rows * g.S_cap * g.WPK * sizeof(float));
     w.list_idx = take(rows * g.l_pad * sizeof(int32_t));
