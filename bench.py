@@ -44,7 +44,44 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", action="store_true",
+                    help="run a small case once (no timing) for ncu captures: refresh step, "
+                         "two reuse steps and one dense call")
+    ap.add_argument("--profile-batch", type=int, default=4)
     return ap.parse_args()
+
+
+def run_profile_case(args):
+    """The case the profiles/ captures use: the workload at a smaller batch
+    (inputs still larger than L2), steps 0..2 and one dense call."""
+    from sparse_decode_attention_saga_b200 import _lib
+    from sparse_decode_attention_saga_b200.decoder import AtopNDecoder
+    w = CONFIGS[args.config].scaled(batch=args.profile_batch)
+    K, V = make_cache(w, args.seed, "cuda")
+    qs = make_queries(w, args.seed, "cuda", steps=3)
+    dec = AtopNDecoder.for_workload(w)
+    for t in range(3):
+        dec.step(t, qs[t], K, V)
+    dec.dense(qs[0], K, V)
+    torch.cuda.synchronize()
+    assert dec.error() == _lib.SAGA_OK
+    return 0
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per launch of the fused kernel from the committed ncu record,
+    or None if the record is for another workload or the kernel sources have
+    changed since the counters were taken."""
+    import hashlib
+    root = os.path.dirname(os.path.abspath(__file__))
+    path = os.path.join(root, "profiles", f"traffic_qk_stream_select_{workload}.json")
+    try:
+        rec = json.load(open(path))
+        h = hashlib.sha256(b"".join(open(os.path.join(root, p), "rb").read()
+                                    for p in rec["sources"])).hexdigest()
+        return float(rec["bytes_per_launch"]) if h == rec["sources_sha256"] else None
+    except Exception:
+        return None
 
 
 def peaks():
@@ -346,7 +383,7 @@ def run_ours(args, world, rank, local):
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "bytes_per_launch": kern_bytes, "us_per_launch": kern_us,
-                     "traffic": None},
+                     "traffic": measured_traffic(w.name)},
         "step_roofline": {"what": "reuse step (fused kernel + gather + combine) vs ideal bytes "
                                   "K + distinct kept V rows + q/tau/out",
                           "ideal_bytes": step_ideal, "us": us_reuse,
@@ -371,6 +408,8 @@ def main():
     args = parse()
     world, rank, local = dist_setup(args)
     try:
+        if args.profile_case:
+            return run_profile_case(args)
         if args.impl == "reference":
             return run_reference(args, world, rank)
         return run_ours(args, world, rank, local)

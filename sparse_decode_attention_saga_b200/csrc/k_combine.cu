@@ -68,7 +68,7 @@ __device__ void fallback_row(const CombineArgs& a, long long row, float m_star, 
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const float s = acc[0][nt][2 * h + e] * g.scale;
+                    const float s = __fmul_rn(acc[0][nt][2 * h + e], g.scale);
                     const int pos = j0 + gq + 8 * h;
                     if (nt == nti && 2 * tq + e == col && pos < g.l && s == m_star) match = true;
                 }

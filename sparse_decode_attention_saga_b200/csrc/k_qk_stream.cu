@@ -15,9 +15,10 @@
 // tensor cores (qk_tile.cuh), then
 //   kStreamLogits: stores them to the logits array (refresh steps), or
 //   kStreamSelect: compares them with the per-(batch, query head) thresholds,
-//     ballots the kept entries and appends (position, logit) to per-(row,
-//     CTA slot, warp) lists in ascending position order, and records the
-//     count and the maximum logit seen (for the empty-set fallback).
+//     appends the kept (position, logit) pairs to per-(row, CTA slot, warp)
+//     lists (offsets from a shuffle scan over the lanes sharing a head), and
+//     records the count and the maximum logit seen (for the empty-set
+//     fallback).
 // Logits never reach device memory on the select path.
 #include "qk_tile.cuh"
 #include "saga_kernels.h"
@@ -26,6 +27,21 @@ namespace saga {
 
 namespace {
 
+// Smallest fp32 x with fl(x * scale) >= tau.  fl(x * scale) is monotone in x,
+// so "x >= raw_threshold(tau, scale)" decides exactly what "fl(x * scale) >=
+// tau" decides, with one compare on the raw tensor-core accumulator.  The
+// start fl(tau / scale) is within two ulps of the boundary.
+__device__ __forceinline__ float raw_threshold(float tau, float scale) {
+    float x = __fdiv_rn(tau, scale);
+    if (!(x == x)) return x;  // NaN threshold: nothing compares >= it
+    for (int i = 0; i < 4 && __fmul_rn(x, scale) >= tau; ++i) {
+        const float below = nextafterf(x, -kInf);
+        if (__fmul_rn(below, scale) < tau) break;
+        x = below;
+    }
+    for (int i = 0; i < 4 && __fmul_rn(x, scale) < tau; ++i) x = nextafterf(x, kInf);
+    return x;
+}
 
 template <int D, int NT, int MODE>
 __global__ void __launch_bounds__(kStreamThreads, 2)
@@ -105,6 +121,8 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
     QFrag<D, NT> qf;
     float tau[NT][2], mall[NT][2];
     int cnt[NT][2];
+    int32_t* lidx[NT][2];  // this warp's kept-position list of each head column
+    float* lsv[NT][2];     // ... and the matching logits
     int cur_bb = -1, slot = 0;
     long long sub_base = 0;
 
@@ -121,9 +139,13 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int hl = nt * 8 + 2 * tq + e;
-                    tau[nt][e] = hl < G ? __ldg(a.thresh + bb * g.hq + kh * G + hl) : kInf;
+                    const int hc = hl < G ? hl : 0;
+                    const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + hc;
+                    tau[nt][e] = hl < G ? raw_threshold(__ldg(a.thresh + row), scale) : kInf;
                     mall[nt][e] = -kInf;
                     cnt[nt][e] = 0;
+                    lidx[nt][e] = a.list_idx + row * g.l_pad + sub_base;
+                    lsv[nt][e] = a.list_s + row * g.l_pad + sub_base;
                 }
         }
     };
@@ -134,10 +156,11 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-                float m = mall[nt][e];
+                float m = mall[nt][e];  // raw accumulator max; scaling is monotone
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                m = __fmul_rn(m, scale);
                 const int hl = nt * 8 + 2 * tq + e;
                 if (gq == 0 && hl < G) {
                     const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + hl;
@@ -148,13 +171,108 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
             }
     };
 
+    // Tile epilogue: logits store, or compare + list append, for the tile
+    // whose (unscaled) accumulators are x, in the current segment.
+    auto epilogue = [&](float (&x)[MBW][NT][4], int tl_e) {
+            const int pos0 = tl_e * g.P + mb0 * 16 + gq;
+            const bool full_tile = (tl_e + 1) * g.P <= g.l;  // every position of the tile is valid
+            if (MODE == kStreamLogits) {
+#pragma unroll
+                for (int mbi = 0; mbi < MBW; ++mbi)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int pos = pos0 + mbi * 16 + 8 * h;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int hl = nt * 8 + 2 * tq + e;
+                                if ((full_tile || pos < g.l) && hl < G)
+                                    a.logits[(static_cast<size_t>(cur_bb) * g.hq + kh * G + hl) * g.l + pos] =
+                                        __fmul_rn(x[mbi][nt][2 * h + e], scale);
+                            }
+                    }
+            } else {
+                // Per n-tile: a bitmask of this thread's kept values (2 heads x
+                // 2*MBW positions), then one segmented scan over the 8 lanes that
+                // share each head (lanes tq, tq+4, ...) gives every thread its
+                // offset in the (row, slot, warp) lists; both heads' counts travel
+                // packed in one word.  The list order is (tile, lane, value):
+                // deterministic, which is all the gather kernel needs.
+                constexpr int HB = 2 * MBW;  // values per head per thread and tile
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    uint32_t km = 0u;
+#pragma unroll
+                    for (int mbi = 0; mbi < MBW; ++mbi)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int pos = pos0 + mbi * 16 + 8 * h;
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                // raw compare (tau holds the raw threshold); head
+                                // columns past G have tau = +inf and are never
+                                // reported, so only the position needs checking
+                                const float v = x[mbi][nt][2 * h + e];
+                                if (full_tile || pos < g.l) {
+                                    mall[nt][e] = fmaxf(mall[nt][e], v);
+                                    if (v >= tau[nt][e]) km |= 1u << (e * HB + mbi * 2 + h);
+                                }
+                            }
+                        }
+                    if (__any_sync(0xffffffffu, km != 0u)) {
+                        const uint32_t mine = static_cast<uint32_t>(__popc(km & ((1u << HB) - 1u))) |
+                                              (static_cast<uint32_t>(__popc(km >> HB)) << 16);
+                        uint32_t inc = mine;
+#pragma unroll
+                        for (int d = 4; d < 32; d <<= 1) {
+                            const uint32_t x = __shfl_up_sync(0xffffffffu, inc, d);
+                            if (lane >= d) inc += x;
+                        }
+                        const uint32_t tot = __shfl_sync(0xffffffffu, inc, 28 + tq);
+                        if (km) {
+                            const uint32_t excl = inc - mine;
+                            int o0 = cnt[nt][0] + static_cast<int>(excl & 0xffffu);
+                            int o1 = cnt[nt][1] + static_cast<int>(excl >> 16);
+#pragma unroll
+                            for (int mbi = 0; mbi < MBW; ++mbi)
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const int pos = pos0 + mbi * 16 + 8 * h;
+                                    if (km & (1u << (mbi * 2 + h))) {
+                                        lidx[nt][0][o0] = pos;
+                                        lsv[nt][0][o0] = __fmul_rn(x[mbi][nt][2 * h], scale);
+                                        ++o0;
+                                    }
+                                    if (km & (1u << (HB + mbi * 2 + h))) {
+                                        lidx[nt][1][o1] = pos;
+                                        lsv[nt][1][o1] = __fmul_rn(x[mbi][nt][2 * h + 1], scale);
+                                        ++o1;
+                                    }
+                                }
+                        }
+                        cnt[nt][0] += static_cast<int>(tot & 0xffffu);
+                        cnt[nt][1] += static_cast<int>(tot >> 16);
+                    }
+                }
+            }
+    };
+
+    // Software pipeline: tile k's mma runs (and its stage is released) before
+    // tile k-1's epilogue, so a stage is handed back as soon as its data has
+    // been read and the epilogue never delays the ring.
     bool ok = true;
     int bb = static_cast<int>(t0 / g.tiles);
     int tl = static_cast<int>(t0 - static_cast<long long>(bb) * g.tiles);
     int st = 0;
     uint32_t phase = 0;
+    float acc_prev[MBW][NT][4];
+    int tl_prev = 0;
+    bool have_prev = false;
     for (int k = 0; k < ntile; ++k) {
         if (bb != cur_bb) {
+            if (have_prev) epilogue(acc_prev, tl_prev);
+            have_prev = false;
             if (cur_bb >= 0) end_segment(cur_bb);
             begin_segment(bb);
             cur_bb = bb;
@@ -172,45 +290,21 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
             st = 0;
             phase ^= 1;
         }
-
-        const int pos0 = tl * g.P + mb0 * 16 + gq;
+        if (have_prev) epilogue(acc_prev, tl_prev);
 #pragma unroll
         for (int mbi = 0; mbi < MBW; ++mbi)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int pos = pos0 + mbi * 16 + 8 * h;
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int hl = nt * 8 + 2 * tq + e;
-                        const bool valid = pos < g.l && hl < G;
-                        const float s = acc[mbi][nt][2 * h + e] * scale;
-                        const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + hl;
-                        if (MODE == kStreamLogits) {
-                            if (valid) a.logits[row * g.l + pos] = s;
-                        } else {
-                            if (valid) mall[nt][e] = fmaxf(mall[nt][e], s);
-                            const bool kept = valid && s >= tau[nt][e];
-                            const uint32_t ball = __ballot_sync(0xffffffffu, kept);
-                            if (ball) {
-                                const uint32_t grp = ball & (0x11111111u << tq);
-                                if (kept) {
-                                    const int off = cnt[nt][e] + __popc(grp & lanemask_lt());
-                                    const size_t at = row * g.l_pad + sub_base + off;
-                                    a.list_idx[at] = pos;
-                                    a.list_s[at] = s;
-                                }
-                                cnt[nt][e] += __popc(grp);
-                            }
-                        }
-                    }
-            }
+                for (int e = 0; e < 4; ++e) acc_prev[mbi][nt][e] = acc[mbi][nt][e];
+        tl_prev = tl;
+        have_prev = true;
         if (++tl == g.tiles) {
             tl = 0;
             ++bb;
         }
     }
+    if (have_prev && ok) epilogue(acc_prev, tl_prev);
     if (cur_bb >= 0) end_segment(cur_bb);
     if (!ok && lane == 0) raise_device_error(a.err, kErrTimeout);
 }
