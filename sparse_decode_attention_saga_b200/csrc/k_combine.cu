@@ -20,7 +20,7 @@ namespace saga {
 
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
 template <int D, int NT>
@@ -95,6 +95,7 @@ template <int D, int NT>
 __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a) {
     __shared__ float red[3][kWarps];
     __shared__ int red_c[kWarps];
+    __shared__ float red_o[kWarps][D];
     __shared__ __align__(1024) uint8_t kbuf[16 * D * 2];
 
     const Geometry& g = a.g;
@@ -159,14 +160,30 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a) 
     for (int w = 0; w < kWarps; ++w) lsum += red[2][w];
     const float inv = 1.f / lsum;
 
-    for (int c = tid; c < D; c += kThreads) {
-        float o = 0.f;
-        for (int r = 0; r < R; ++r) {
-            const float* rec = recs + static_cast<size_t>(r) * g.rec;
-            const float m = rec[0];
-            if (m > -kInf) o += rec[kRecHeader + c] * __expf(m - M);
+    // Records are spread over the warps (warp w sums records w, w+4, ...;
+    // lane owns D/32 columns), so the loads of different records are in
+    // flight together; the warps' partial sums are then added in a fixed order.
+    constexpr int CPL = D / 32;
+    float o[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) o[c] = 0.f;
+    for (int r = warp; r < R; r += kWarps) {
+        const float* rec = recs + static_cast<size_t>(r) * g.rec;
+        const float m = rec[0];
+        if (m > -kInf) {
+            const float wgt = __expf(m - M);
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) o[c] = fmaf(rec[kRecHeader + lane * CPL + c], wgt, o[c]);
         }
-        out_row[c] = o * inv;
+    }
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) red_o[warp][lane * CPL + c] = o[c];
+    __syncthreads();
+    for (int c = tid; c < D; c += kThreads) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) v += red_o[w][c];
+        out_row[c] = v * inv;
     }
     if (tid == 0 && a.sel_cnt) a.sel_cnt[row] = cnt;
 }

@@ -30,6 +30,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kMinShare = 128;  // kept entries per CTA at least
 #ifndef SAGA_GATHER_INFLIGHT
 #define SAGA_GATHER_INFLIGHT 4
 #endif
@@ -48,7 +49,7 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     constexpr int UNROLL = 8;
     constexpr int MBW = 128 / D;
 
-    extern __shared__ int table[];     // pre[max_lists + 1], start[max_lists]
+    extern __shared__ int table[];     // pre, start, slot_pos, slot_len
     __shared__ float red_m[kWarps];
     __shared__ float red_l[kWarps];
     __shared__ float red_o[kWarps][D];
@@ -62,8 +63,10 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     const int bb = static_cast<int>(row / g.hq);
     const int i = static_cast<int>(row - static_cast<long long>(bb) * g.hq);
     const int vh = i * g.hv / g.hq;
-    int* pre = table;                       // exclusive prefix of list counts; pre[nl] = total
-    int* start = table + a.max_lists + 1;   // list start inside the row's list region
+    int* pre = table;                        // exclusive prefix of list counts; pre[nl] = total
+    int* start = table + a.max_lists + 1;    // list start inside the row's list region
+    int* slot_pos = start + a.max_lists;     // per slot: first position of its segment
+    int* slot_len = slot_pos + a.max_slots;  // per slot: capacity of each warp's list
 
     // ---- list table of the row
     float m_all = -kInf;
@@ -83,26 +86,33 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
         const int c_first = cta_of_tile(x0, T, a.C);
         const int slots = cta_of_tile(x0 + g.tiles - 1, T, a.C) - c_first + 1;
         nl = slots * g.WPK;  // <= max_lists (checked by the host)
-        const int per = (nl + kThreads - 1) / kThreads;
-        const int j0 = min(nl, tid * per), j1 = min(nl, j0 + per);
-        int run = 0;
-        float mloc = -kInf;
-        for (int j = j0; j < j1; ++j) {
-            const int slot = j / g.WPK, u = j - slot * g.WPK;
-            const int c = c_first + slot;
+        // per-slot position offset and tile count of the streaming CTA's segment
+        for (int sl = tid; sl < slots; sl += kThreads) {
+            const int c = c_first + sl;
             const long long t0 = cta_tile_begin(T, a.C, c), t1 = cta_tile_begin(T, a.C, c + 1);
             const long long s0 = t0 > x0 ? t0 : x0;
             const long long s1 = t1 < x0 + g.tiles ? t1 : x0 + g.tiles;
-            // a list never holds more entries than its warp's positions
-            const int cap = static_cast<int>((s1 - s0) * MBW * 16);
-            const size_t at = (static_cast<size_t>(row) * g.S_cap + slot) * g.WPK + u;
-            const int cu = a.seg_cnt[at];
-            start[j] = static_cast<int>((s0 - x0) * g.P +
-                                        static_cast<long long>(u) * (s1 - s0) * MBW * 16);
-            pre[j] = cu < 0 ? 0 : (cu > cap ? cap : cu);  // counts for now
-            run += pre[j];
-            mloc = fmaxf(mloc, a.seg_mall[at]);
+            slot_pos[sl] = static_cast<int>((s0 - x0) * g.P);
+            slot_len[sl] = static_cast<int>((s1 - s0) * MBW * 16);  // entries a warp can hold
         }
+        __syncthreads();
+        // counts (coalesced reads), clamped to each list's capacity
+        const size_t rbase = static_cast<size_t>(row) * g.S_cap * g.WPK;
+        float mloc = -kInf;
+        for (int j = tid; j < nl; j += kThreads) {
+            const int cu = a.seg_cnt[rbase + j];
+            const int sl = j / g.WPK;
+            const int cap = slot_len[sl];
+            start[j] = slot_pos[sl] + (j - sl * g.WPK) * cap;
+            pre[j] = cu < 0 ? 0 : (cu > cap ? cap : cu);
+            mloc = fmaxf(mloc, a.seg_mall[rbase + j]);
+        }
+        __syncthreads();
+        // exclusive scan: each thread owns a run of consecutive lists
+        const int per = (nl + kThreads - 1) / kThreads;
+        const int j0 = min(nl, tid * per), j1 = min(nl, j0 + per);
+        int run = 0;
+        for (int j = j0; j < j1; ++j) run += pre[j];
         int inc = run;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -133,8 +143,12 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
         __syncthreads();
     }
     const int total = pre[nl];
-    const int e0 = static_cast<int>(static_cast<long long>(total) * part / a.parts);
-    const int e1 = static_cast<int>(static_cast<long long>(total) * (part + 1) / a.parts);
+    // Shares of at least kMinShare entries: with few kept entries per row most
+    // of the launched parts stay empty (their records say so) instead of each
+    // paying a CTA's fixed cost for a handful of rows.
+    const int parts = max(1, min(a.parts, (total + kMinShare - 1) / kMinShare));
+    const int e0 = part < parts ? static_cast<int>(static_cast<long long>(total) * part / parts) : total;
+    const int e1 = part < parts ? static_cast<int>(static_cast<long long>(total) * (part + 1) / parts) : total;
     const int n = e1 - e0;
     // each warp owns a contiguous sub-share and needs no block barrier
     const int w0 = e0 + static_cast<int>(static_cast<long long>(n) * warp / kWarps);
@@ -241,13 +255,13 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
 
 }  // namespace
 
-size_t gather_smem_bytes(int max_lists) {
-    return (2 * static_cast<size_t>(max_lists) + 1) * sizeof(int);
+size_t gather_smem_bytes(int max_lists, int max_slots) {
+    return (2 * static_cast<size_t>(max_lists) + 1 + 2 * static_cast<size_t>(max_slots)) * sizeof(int);
 }
 
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
     const dim3 grid(a.parts, static_cast<unsigned>(static_cast<long long>(a.g.b) * a.g.hq));
-    const size_t smem = gather_smem_bytes(a.max_lists);
+    const size_t smem = gather_smem_bytes(a.max_lists, a.max_slots);
     if (smem > static_cast<size_t>(kGatherMaxSmem)) return cudaErrorInvalidValue;
     if (a.g.d == 64) {
         static const cudaError_t attr = cudaFuncSetAttribute(

@@ -31,6 +31,7 @@ namespace {
 #endif
 constexpr int kStreamStages = SAGA_STREAM_STAGES;
 constexpr int kStreamCtasPerSm = SAGA_STREAM_CTAS_PER_SM;
+constexpr long long kMinTilesPerCta = 4;
 constexpr int kMaxDevices = 64;
 
 std::atomic<uint64_t> g_launches{0};
@@ -153,6 +154,10 @@ int stream_ctas(const Geometry& g, const DeviceInfo& dev, int per_sm = kStreamCt
     const long long T = static_cast<long long>(g.b) * g.tiles;
     long long c = static_cast<long long>(dev.sms) * per_sm;
     if (c > kMaxCtas) c = kMaxCtas;
+    // at least kMinTilesPerCta tiles each: a CTA's pipeline start costs a few
+    // microseconds, and every CTA adds a partial-record slot to each row
+    const long long by_work = (T + kMinTilesPerCta - 1) / kMinTilesPerCta;
+    if (c > by_work) c = by_work;
     if (c > T) c = T;
     int C = static_cast<int>(c < 1 ? 1 : c);
     while (C > 1 && max_slots(g, T, C) > g.S_cap) --C;
@@ -332,6 +337,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         ga.mode = kListContiguous;
         ga.parts = gather_parts(g, dev);
         ga.max_lists = 1;
+        ga.max_slots = 1;
         ga.v = v;
         ga.idx = sa.idx;
         ga.list_s = sa.s;
@@ -378,8 +384,9 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     ga.mode = kListSegments;
     ga.C = a.C;
     ga.parts = gather_parts(g, dev);
-    ga.max_lists = max_slots(g, static_cast<long long>(g.b) * g.tiles, a.C) * g.WPK;
-    if (gather_smem_bytes(ga.max_lists) > static_cast<size_t>(kGatherMaxSmem))
+    ga.max_slots = max_slots(g, static_cast<long long>(g.b) * g.tiles, a.C);
+    ga.max_lists = ga.max_slots * g.WPK;
+    if (gather_smem_bytes(ga.max_lists, ga.max_slots) > static_cast<size_t>(kGatherMaxSmem))
         return SAGA_ERR_UNSUPPORTED;
     ga.v = v;
     ga.list_idx = a.list_idx;

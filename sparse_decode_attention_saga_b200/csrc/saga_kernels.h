@@ -76,6 +76,7 @@ struct GatherArgs {
     int parts;      // CTAs per row (each takes an equal share of the row's entries)
     int C;          // kListSegments: grid of the fused kernel
     int max_lists;  // lists per row at most (kListSegments: slots * WPK; else 1)
+    int max_slots;  // kListSegments: streaming-CTA slots per row at most; else 1
     const void* v;
     const int32_t* idx;       // kListContiguous: positions [rows][l]
     const int32_t* cnt;       // kListContiguous: counts [rows]
@@ -86,7 +87,7 @@ struct GatherArgs {
     const float* seg_mall;
     float* records;
 };
-size_t gather_smem_bytes(int max_lists);
+size_t gather_smem_bytes(int max_lists, int max_slots);
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream);
 
 // Dense flash-decoding kernel (K and V streamed) -> partial records.
