@@ -154,6 +154,14 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
 int saga_topn_refresh_noalloc(const saga_dims* dims, int32_t N, const float* logits_in,
                               float* thresh_out, saga_stream_t stream);
 
+/* Failure-path self-test (the paper has no counterpart): one CTA waits, with
+ * the bounded wait every pipelined kernel uses, on a barrier that nothing
+ * completes; after limit_us microseconds (1 .. 1000000) it gives up, sets the
+ * workspace's sticky timeout flag and returns.  Lets a test check that a
+ * wait which runs out surfaces as SAGA_ERR_TIMEOUT from saga_workspace_error
+ * and leaves the context usable.  Only the first 256 bytes of ws are used. */
+int saga_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us, saga_stream_t stream);
+
 /* Enqueue a zeroing of the workspace (sticky flags included). */
 int saga_workspace_reset(void* ws, size_t ws_bytes, saga_stream_t stream);
 

@@ -27,6 +27,7 @@ EXPORTS = (
     "saga_workspace_bytes", "saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
     "saga_workspace_reset", "saga_workspace_error", "saga_status_string", "saga_launch_count",
     "saga_set_kernel_events", "saga_version", "saga_topn_refresh_noalloc",
+    "saga_selftest_wait_timeout",
 )
 
 
@@ -66,6 +67,8 @@ def load(path: str | None = None):
         lib.saga_atopn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, SZ, P]
         lib.saga_topn_refresh_noalloc.argtypes = [D, I32, P, P, P]
         lib.saga_topn_refresh_noalloc.restype = ctypes.c_int
+        lib.saga_selftest_wait_timeout.argtypes = [P, SZ, ctypes.c_uint32, P]
+        lib.saga_selftest_wait_timeout.restype = ctypes.c_int
         lib.saga_workspace_reset.argtypes = [P, SZ, P]
         lib.saga_workspace_error.argtypes = [P, SZ, P]
         lib.saga_status_string.argtypes = [ctypes.c_int]
@@ -139,6 +142,13 @@ def topn_refresh_noalloc(d, N, logits_in, thresh_out, stream=None) -> None:
     st = load().saga_topn_refresh_noalloc(ctypes.byref(d), int(N), _ptr(logits_in),
                                           _ptr(thresh_out), _stream(stream))
     _check("saga_topn_refresh_noalloc", st)
+
+
+def selftest_wait_timeout(ws, limit_us: int, stream=None) -> None:
+    """Make a bounded device wait run out on purpose (sets the timeout flag)."""
+    _check("saga_selftest_wait_timeout",
+           load().saga_selftest_wait_timeout(_ptr(ws), ws.numel() * ws.element_size(),
+                                             int(limit_us), _stream(stream)))
 
 
 def workspace_reset(ws, stream=None) -> None:
