@@ -32,6 +32,8 @@ SHAPES = [
     ("g16_two_ntiles", 1, 16, 1, 16, 64, 1100, None),
     ("g3_d128", 3, 6, 2, 2, 128, 4097, None),
     ("saga_1_8", 2, 16, 1, 8, 64, 3000, None),
+    # h_q > 32: the reuse step takes the list path (compare kernel, gather, combine)
+    ("hq64_lists", 2, 64, 4, 8, 64, 1500, None),
 ]
 
 
