@@ -180,8 +180,14 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
                 if (pre[mid] <= e) lo = mid; else hi = mid - 1;
             }
             const long long at = row_base + start[lo] + (e - pre[lo]);
-            pos = __ldg((a.mode == kListContiguous ? a.idx : a.list_idx) + at);
-            s = __ldg(a.list_s + at);
+            if (a.mode == kListContiguous) {
+                pos = __ldg(a.idx + at);
+                s = __ldg(a.list_s + at);
+            } else {
+                const int2 ps = __ldg(a.seg_list + at);
+                pos = ps.x;
+                s = __int_as_float(ps.y);
+            }
         }
     };
     int nxt_pos;

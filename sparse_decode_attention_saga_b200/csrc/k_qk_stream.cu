@@ -121,8 +121,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
     QFrag<D, NT> qf;
     float tau[NT][2], mall[NT][2];
     int cnt[NT][2];
-    int32_t* lidx[NT][2];  // this warp's kept-position list of each head column
-    float* lsv[NT][2];     // ... and the matching logits
+    int2* lst[NT][2];  // this warp's kept (position, logit) list of each head column
     int cur_bb = -1, slot = 0;
     long long sub_base = 0;
 
@@ -144,8 +143,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
                     tau[nt][e] = hl < G ? raw_threshold(__ldg(a.thresh + row), scale) : kInf;
                     mall[nt][e] = -kInf;
                     cnt[nt][e] = 0;
-                    lidx[nt][e] = a.list_idx + row * g.l_pad + sub_base;
-                    lsv[nt][e] = a.list_s + row * g.l_pad + sub_base;
+                    lst[nt][e] = a.list + row * g.l_pad + sub_base;
                 }
         }
     };
@@ -240,13 +238,13 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
                                 for (int h = 0; h < 2; ++h) {
                                     const int pos = pos0 + mbi * 16 + 8 * h;
                                     if (km & (1u << (mbi * 2 + h))) {
-                                        lidx[nt][0][o0] = pos;
-                                        lsv[nt][0][o0] = __fmul_rn(x[mbi][nt][2 * h], scale);
+                                        lst[nt][0][o0] = make_int2(
+                                            pos, __float_as_int(__fmul_rn(x[mbi][nt][2 * h], scale)));
                                         ++o0;
                                     }
                                     if (km & (1u << (HB + mbi * 2 + h))) {
-                                        lidx[nt][1][o1] = pos;
-                                        lsv[nt][1][o1] = __fmul_rn(x[mbi][nt][2 * h + 1], scale);
+                                        lst[nt][1][o1] = make_int2(
+                                            pos, __float_as_int(__fmul_rn(x[mbi][nt][2 * h + 1], scale)));
                                         ++o1;
                                     }
                                 }

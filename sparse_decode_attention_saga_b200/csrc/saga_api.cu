@@ -368,8 +368,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     a.stages = kStreamStages;
     a.q = q;
     a.thresh = thresh;
-    a.list_idx = ws_at<int32_t>(ws, L.list_idx);
-    a.list_s = ws_at<float>(ws, L.list_s);
+    a.list = ws_at<int2>(ws, L.list_idx);  // spans the list_idx and list_s regions
     a.seg_cnt = ws_at<int32_t>(ws, L.seg_cnt);
     a.seg_mall = ws_at<float>(ws, L.seg_mall);
     a.err = err;
@@ -389,8 +388,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     if (gather_smem_bytes(ga.max_lists, ga.max_slots) > static_cast<size_t>(kGatherMaxSmem))
         return SAGA_ERR_UNSUPPORTED;
     ga.v = v;
-    ga.list_idx = a.list_idx;
-    ga.list_s = a.list_s;
+    ga.seg_list = a.list;
     ga.seg_cnt = a.seg_cnt;
     ga.seg_mall = a.seg_mall;
     ga.records = records;

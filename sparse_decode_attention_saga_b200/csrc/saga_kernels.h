@@ -21,8 +21,7 @@ struct StreamArgs {
     const void* q;
     const float* thresh;
     float* logits;
-    int32_t* list_idx;
-    float* list_s;
+    int2* list;  // kept (position, logit bits) pairs, per (row, slot, warp) segment
     int32_t* seg_cnt;
     float* seg_mall;
     uint32_t* err;
@@ -81,8 +80,8 @@ struct GatherArgs {
     const int32_t* idx;       // kListContiguous: positions [rows][l]
     const int32_t* cnt;       // kListContiguous: counts [rows]
     const float* rowmax;      // kListContiguous: largest logit per row [rows]
-    const int32_t* list_idx;  // kListSegments: positions [rows][l_pad]
-    const float* list_s;      // logits of the listed entries (row stride l or l_pad)
+    const float* list_s;      // kListContiguous: logits of the listed entries [rows][l]
+    const int2* seg_list;     // kListSegments: (position, logit bits) pairs [rows][l_pad]
     const int32_t* seg_cnt;
     const float* seg_mall;
     float* records;

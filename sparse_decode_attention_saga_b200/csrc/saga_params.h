@@ -72,8 +72,8 @@ struct WsLayout {
     size_t rowmax;    // float  [b*hq]
     size_t seg_cnt;   // int32  [b*hq][S_cap][WPK]
     size_t seg_mall;  // float  [b*hq][S_cap][WPK]
-    size_t list_idx;  // int32  [b*hq][l_pad]
-    size_t list_s;    // float  [b*hq][l_pad]
+    size_t list_idx;  // int32  [b*hq][l_pad]; with list_s also the int2 [b*hq][l_pad]
+    size_t list_s;    // float  [b*hq][l_pad]   (position, logit) pairs of the fused path
     size_t logits;    // float  [b*hq][l]
     size_t total;
 };
