@@ -98,6 +98,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a) 
     __shared__ float red_o[kWarps][D];
     __shared__ __align__(1024) uint8_t kbuf[16 * D * 2];
 
+    pdl_wait();  // the partial records come from the previous kernel
     const Geometry& g = a.g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long row = blockIdx.x;
@@ -193,12 +194,12 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a) 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
     const unsigned rows = static_cast<unsigned>(static_cast<long long>(a.g.b) * a.g.hq);
     const int d = a.g.d, nt = a.g.NT;
-    if (d == 64 && nt == 1) combine_kernel<64, 1><<<rows, kThreads, 0, stream>>>(a);
-    else if (d == 64 && nt == 2) combine_kernel<64, 2><<<rows, kThreads, 0, stream>>>(a);
-    else if (d == 128 && nt == 1) combine_kernel<128, 1><<<rows, kThreads, 0, stream>>>(a);
-    else if (d == 128 && nt == 2) combine_kernel<128, 2><<<rows, kThreads, 0, stream>>>(a);
-    else return cudaErrorInvalidValue;
-    return cudaGetLastError();
+    const dim3 grid(rows), block(kThreads);
+    if (d == 64 && nt == 1) return launch_dependent(combine_kernel<64, 1>, grid, block, 0, stream, a);
+    if (d == 64 && nt == 2) return launch_dependent(combine_kernel<64, 2>, grid, block, 0, stream, a);
+    if (d == 128 && nt == 1) return launch_dependent(combine_kernel<128, 1>, grid, block, 0, stream, a);
+    if (d == 128 && nt == 2) return launch_dependent(combine_kernel<128, 2>, grid, block, 0, stream, a);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace saga

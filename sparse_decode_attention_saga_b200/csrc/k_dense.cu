@@ -53,6 +53,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_trigger();  // the combine kernel may be scheduled behind this grid
 
     const long long T = static_cast<long long>(g.b) * g.tiles;
     const int C = a.C, c = blockIdx.x;

@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     __shared__ int red_i[kWarps];
     __shared__ long long row_base;
 
+    pdl_wait();     // lists, counts and maxima come from the previous kernel
+    pdl_trigger();
     const Geometry& g = a.g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long row = blockIdx.y;
@@ -273,14 +275,13 @@ cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
         static const cudaError_t attr = cudaFuncSetAttribute(
             gather_pv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem);
         if (attr != cudaSuccess) return attr;
-        gather_pv_kernel<64><<<grid, kThreads, smem, stream>>>(a);
+        return launch_dependent(gather_pv_kernel<64>, grid, dim3(kThreads), smem, stream, a);
     } else {
         static const cudaError_t attr = cudaFuncSetAttribute(
             gather_pv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem);
         if (attr != cudaSuccess) return attr;
-        gather_pv_kernel<128><<<grid, kThreads, smem, stream>>>(a);
+        return launch_dependent(gather_pv_kernel<128>, grid, dim3(kThreads), smem, stream, a);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace saga

@@ -67,6 +67,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_trigger();  // the gather kernel may be scheduled behind this grid
 
     const long long T = static_cast<long long>(g.b) * g.tiles;
     const int C = a.C, c = blockIdx.x;

@@ -60,6 +60,8 @@ __global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a)
     __shared__ uint32_t warp_tot[kThreads / 32];
     __shared__ int is_last;
 
+    pdl_wait();  // logits, histograms and the previous pass's state
+    pdl_trigger();
     const int tid = threadIdx.x;
     const long long row = blockIdx.y;
     const int chunk = blockIdx.x;
@@ -158,16 +160,21 @@ __global__ void fill_kernel(float* p, long long n, float value) {
 cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream) {
     const dim3 grid(a.chunks, static_cast<unsigned>(a.rows));
     const bool vec = (a.l % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.logits) & 15u) == 0);
+    const dim3 block(kThreads);
+    // pass 0 follows the histogram clear (an ordinary launch); passes 1 and 2
+    // may be scheduled while the pass before them drains
     if (vec) {
-        radix_pass_kernel<0, 4><<<grid, kThreads, 0, stream>>>(a);
-        radix_pass_kernel<1, 4><<<grid, kThreads, 0, stream>>>(a);
-        radix_pass_kernel<2, 4><<<grid, kThreads, 0, stream>>>(a);
-    } else {
-        radix_pass_kernel<0, 1><<<grid, kThreads, 0, stream>>>(a);
-        radix_pass_kernel<1, 1><<<grid, kThreads, 0, stream>>>(a);
-        radix_pass_kernel<2, 1><<<grid, kThreads, 0, stream>>>(a);
+        radix_pass_kernel<0, 4><<<grid, block, 0, stream>>>(a);
+        cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess) e = launch_dependent(radix_pass_kernel<1, 4>, grid, block, 0, stream, a);
+        if (e == cudaSuccess) e = launch_dependent(radix_pass_kernel<2, 4>, grid, block, 0, stream, a);
+        return e;
     }
-    return cudaGetLastError();
+    radix_pass_kernel<0, 1><<<grid, block, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = launch_dependent(radix_pass_kernel<1, 1>, grid, block, 0, stream, a);
+    if (e == cudaSuccess) e = launch_dependent(radix_pass_kernel<2, 1>, grid, block, 0, stream, a);
+    return e;
 }
 
 cudaError_t launch_fill(float* p, long long n, float value, cudaStream_t stream) {

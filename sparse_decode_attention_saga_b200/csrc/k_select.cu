@@ -35,6 +35,8 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
     __shared__ int round_total;
     __shared__ float red[kWarps];
 
+    pdl_wait();  // the logits and thresholds come from earlier kernels
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long long row = blockIdx.x;
     const float* src = a.logits + row * a.l;
@@ -136,11 +138,9 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
 
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream) {
     const bool vec = (a.l % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.logits) & 15u) == 0);
-    if (vec)
-        select_compact_kernel<4><<<static_cast<unsigned>(a.rows), kThreads, 0, stream>>>(a);
-    else
-        select_compact_kernel<1><<<static_cast<unsigned>(a.rows), kThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    const dim3 grid(static_cast<unsigned>(a.rows)), block(kThreads);
+    return vec ? launch_dependent(select_compact_kernel<4>, grid, block, 0, stream, a)
+               : launch_dependent(select_compact_kernel<1>, grid, block, 0, stream, a);
 }
 
 }  // namespace saga

@@ -25,6 +25,19 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
     return t;
 }
 
+// ----------------------------------------------------------------- launch order
+
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may be scheduled while the kernel before it
+// in the stream is still running; pdl_wait() blocks until that kernel has
+// completed and its memory writes are visible, so it must precede every read
+// of the predecessor's results.  pdl_trigger() lets the next kernel of the
+// stream be scheduled early.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- errors
 
 // Sticky device flag at the head of the workspace (read by
