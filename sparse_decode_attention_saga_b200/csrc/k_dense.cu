@@ -4,13 +4,19 @@
 //
 // Split-K (flash-decoding) over the flattened (batch, tile) space, same
 // partition as the streaming kernel.  The producer warp loads each tile's K
-// boxes (128-byte swizzle, read by ldmatrix) and V boxes (plain rows) with
-// TMA; each consumer warp computes the logits of its key head's G query heads
-// for its slice of the tile on tensor cores (the same routine as the sparse
-// path), keeps a running max / sum per head (online softmax), writes the
-// weights to a per-warp scratch, and accumulates weight x value in fp32 on
-// the CUDA cores, each lane owning d/32 output columns.  Every warp writes
-// one partial record per (row, CTA slot); the combine kernel merges them.
+// and V boxes with TMA (128-byte swizzle).  Each consumer warp owns one key
+// head and a slice of the tile's positions:
+//   logits of its G query heads on tensor cores (the same routine as the
+//   sparse path), online softmax per head (running max / sum), and the
+//   weights written to a per-warp scratch as bf16 hi + lo parts
+//   (p = hi + lo to about 16 bits);
+//   the probability-value product also on tensor cores, swap-AB:
+//   O^T (16 head dims x 8 query heads) += V^T (16 dims x 16 positions,
+//   ldmatrix.trans from the swizzled V box) x P^T (16 positions x 8 heads),
+//   once with the hi and once with the lo weights, fp32 accumulators in
+//   registers.  The query heads of one column tile share one value head.
+// Every warp writes one partial record per (row, CTA slot); the combine
+// kernel merges them.
 #include "qk_tile.cuh"
 #include "saga_kernels.h"
 
@@ -18,17 +24,20 @@ namespace saga {
 
 namespace {
 
-constexpr int kPStride = 36;  // floats per head row of the weight scratch (bank spread)
+// bf16 entries per head row of the weight scratch: a warp's positions + 8
+// (the B-fragment reads of the eight heads then hit distinct banks)
+__host__ __device__ constexpr int weight_stride(int d) { return (128 / d) * 16 + 8; }
 
-template <int D, int NT>
+template <int D, int NT, int NCT>
 __global__ void __launch_bounds__(kStreamThreads, 1)
     dense_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                  const DenseArgs a) {
     constexpr int MBW = 128 / D;
     constexpr int DH = D / 64;
-    constexpr int HS = NT * 8;        // head slots per key head
-    constexpr int CPL = D / 32;       // output columns per lane
-    constexpr int ROWS = MBW * 16;    // positions per warp per tile
+    constexpr int HS = NT * 8;         // head slots per key head
+    constexpr int ROWS = MBW * 16;     // positions per warp per tile
+    constexpr int PS = weight_stride(D);
+    constexpr int MT = D / 16;         // 16-dim row tiles of O^T
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -37,8 +46,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     const int stages = a.stages;
     const int vbytes = g.P * g.hv * D * 2;
     const int stage_bytes = kStageBytes + vbytes;
-    float* pbuf_all = reinterpret_cast<float*>(smem + static_cast<size_t>(stages) * stage_bytes);
-    float* abuf_all = pbuf_all + kConsumerWarps * HS * kPStride;
+    uint16_t* pbuf_all = reinterpret_cast<uint16_t*>(smem + static_cast<size_t>(stages) * stage_bytes);
+    float* abuf_all = reinterpret_cast<float*>(pbuf_all + kConsumerWarps * 2 * HS * PS);
     uint64_t* full = reinterpret_cast<uint64_t*>(abuf_all + kConsumerWarps * HS);
     uint64_t* empty = full + stages;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + stages);
@@ -96,21 +105,25 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     const int mb0 = sub * MBW;
     const int gq = lane >> 2, tq = lane & 3;
     const int G = g.G;
-    float* pbuf = pbuf_all + warp * HS * kPStride;
+    uint16_t* pb_hi = pbuf_all + warp * 2 * HS * PS;
+    uint16_t* pb_lo = pb_hi + HS * PS;
     float* abuf = abuf_all + warp * HS;
-    // value-row byte offset of this lane's columns inside a (vh, dh) box row
-    const int vcol_dh = (lane * CPL) / 64;
-    const int vcol_off = ((lane * CPL) % 64) * 2;
-    int vbox[HS];
+
+    // Column tiles of O^T: NCT tiles of 8 head slots.  With two value heads
+    // per key head (VPK = 2) tile ct holds the GV <= 8 query heads of value
+    // head kh*2 + ct; otherwise the G heads of the group's one value head
+    // fill tiles of 8.
+    const int VPK = g.hv > g.hk ? g.hv / g.hk : 1;
+    const int GV = G / VPK;
+    auto head_of = [&](int ct, int n) { return VPK == 2 ? ct * GV + n : ct * 8 + n; };
+    auto head_ok = [&](int ct, int n) { return VPK == 2 ? n < GV : ct * 8 + n < G; };
+    int vh_ct[NCT];
 #pragma unroll
-    for (int hl = 0; hl < HS; ++hl) {
-        const int vh = hl < G ? (kh * G + hl) * g.hv / g.hq : 0;
-        vbox[hl] = kStageBytes + (vh * DH + vcol_dh) * g.P * 128 + vcol_off;
-    }
+    for (int ct = 0; ct < NCT; ++ct) vh_ct[ct] = (kh * G + head_of(ct, 0)) * g.hv / g.hq;
 
     QFrag<D, NT> qf;
     float m_run[NT][2], l_run[NT][2];
-    float o[HS][CPL];
+    float o[MT][NCT][4];  // O^T fragments: dims mt*16 + gq (+8), heads 2tq (+1) of tile ct
     int cur_bb = -1, slot = 0;
 
     auto begin_segment = [&](int bb) {
@@ -124,13 +137,15 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 l_run[nt][e] = 0.f;
             }
 #pragma unroll
-        for (int hl = 0; hl < HS; ++hl)
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-            for (int cc = 0; cc < CPL; ++cc) o[hl][cc] = 0.f;
+            for (int ct = 0; ct < NCT; ++ct)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[mt][ct][e] = 0.f;
     };
 
     auto end_segment = [&](int bb) {
-        // header by the lanes that own each head's softmax state, o by all lanes
+        // header by the lanes that own each head's softmax state
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -146,18 +161,29 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                     rec[3] = m_run[nt][e];
                 }
             }
+        // output columns from the O^T fragments
 #pragma unroll
-        for (int hl = 0; hl < HS; ++hl) {
-            if (hl >= G) break;
-            const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + hl;
-            float* rec =
-                a.records + ((row * g.S_cap + slot) * g.WPK + sub) * static_cast<size_t>(g.rec);
+        for (int ct = 0; ct < NCT; ++ct)
 #pragma unroll
-            for (int cc = 0; cc < CPL; ++cc) rec[kRecHeader + lane * CPL + cc] = o[hl][cc];
-        }
+            for (int e = 0; e < 2; ++e) {
+                if (!head_ok(ct, 2 * tq + e)) continue;
+                const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + head_of(ct, 2 * tq + e);
+                float* rec = a.records +
+                             ((row * g.S_cap + slot) * g.WPK + sub) * static_cast<size_t>(g.rec) + kRecHeader;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    rec[mt * 16 + gq] = o[mt][ct][e];
+                    rec[mt * 16 + gq + 8] = o[mt][ct][2 + e];
+                }
+            }
     };
 
     const uint32_t stage0 = smem_addr(smem);
+    const uint32_t pb_hi_a = smem_addr(pb_hi), pb_lo_a = smem_addr(pb_lo);
+    // ldmatrix.trans addressing: lane -> matrix mi = lane/8 (dims +8 for odd mi,
+    // positions +8 for mi >= 2), row = lane%8 (one position per row)
+    const int ld_pos = (lane >> 4) * 8 + (lane & 7);
+    const int ld_dim = ((lane >> 3) & 1) * 8;
     bool ok = true;
     for (int k = 0; k < ntile; ++k) {
         const long long t = t0 + k;
@@ -178,14 +204,14 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
         float acc[MBW][NT][4];
         qk_mma<D, NT, MBW>(sbase, g.P, kh, mb0, qf, acc, lane);
 
-        // online softmax per head column (2t+e of n-tile nt)
+        // online softmax per head column (2t+e of n-tile nt); weights -> scratch
         const int pos0 = tl * g.P + mb0 * 16 + gq;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 const int hl = nt * 8 + 2 * tq + e;
-                float mt = -kInf;
+                float mt_ = -kInf;
 #pragma unroll
                 for (int mbi = 0; mbi < MBW; ++mbi)
 #pragma unroll
@@ -194,12 +220,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                         const bool valid = pos < g.l && hl < G;
                         const float s = valid ? acc[mbi][nt][2 * h + e] * g.scale : -kInf;
                         acc[mbi][nt][2 * h + e] = s;
-                        mt = fmaxf(mt, s);
+                        mt_ = fmaxf(mt_, s);
                     }
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-                const float m_new = fmaxf(m_run[nt][e], mt);
+                mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 4));
+                mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 8));
+                mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 16));
+                const float m_new = fmaxf(m_run[nt][e], mt_);
                 const bool live = m_new > -kInf;
                 const float alpha = live ? __expf(m_run[nt][e] - m_new) : 1.f;
                 float psum = 0.f;
@@ -210,7 +236,11 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                         const float s = acc[mbi][nt][2 * h + e];
                         const float p = live ? __expf(s - m_new) : 0.f;
                         psum += p;
-                        pbuf[hl * kPStride + mbi * 16 + 8 * h + gq] = p;
+                        const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+                        const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
+                        const int at = hl * PS + mbi * 16 + 8 * h + gq;
+                        pb_hi[at] = __bfloat16_as_ushort(hi);
+                        pb_lo[at] = __bfloat16_as_ushort(lo);
                     }
                 psum += __shfl_xor_sync(0xffffffffu, psum, 4);
                 psum += __shfl_xor_sync(0xffffffffu, psum, 8);
@@ -221,33 +251,67 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
             }
         __syncwarp();
 
-        // o[hl] = alpha * o[hl] + sum_j p[hl][j] * V[j, vh(hl)]
-        const uint8_t* stage_ptr = smem + static_cast<size_t>(st) * stage_bytes;
+        // rescale O^T by each head's alpha, then O^T += V^T P^T (hi and lo)
 #pragma unroll
-        for (int hl = 0; hl < HS; ++hl) {
-            if (hl >= G) break;
-            const float alpha = abuf[hl];
+        for (int ct = 0; ct < NCT; ++ct)
 #pragma unroll
-            for (int cc = 0; cc < CPL; ++cc) o[hl][cc] *= alpha;
-            const uint8_t* vrow = stage_ptr + vbox[hl] + (mb0 * 16) * 128;
+            for (int e = 0; e < 2; ++e) {
+                const float al = head_ok(ct, 2 * tq + e) ? abuf[head_of(ct, 2 * tq + e)] : 1.f;
 #pragma unroll
-            for (int j = 0; j < ROWS; j += 4) {
-                const float4 p4 = *reinterpret_cast<const float4*>(pbuf + hl * kPStride + j);
-                const float pj[4] = {p4.x, p4.y, p4.z, p4.w};
+                for (int mt = 0; mt < MT; ++mt) {
+                    o[mt][ct][e] *= al;
+                    o[mt][ct][2 + e] *= al;
+                }
+            }
+        const int lim = g.l - (tl * g.P + mb0 * 16);  // valid positions of this warp's slice
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint8_t* vp = vrow + (j + jj) * 128;
-                    if (CPL == 2) {
-                        const uint32_t w = *reinterpret_cast<const uint32_t*>(vp);
-                        o[hl][0] = fmaf(pj[jj], bf16_lo(w), o[hl][0]);
-                        o[hl][1] = fmaf(pj[jj], bf16_hi(w), o[hl][1]);
-                    } else {
-                        const uint2 w = *reinterpret_cast<const uint2*>(vp);
-                        o[hl][0] = fmaf(pj[jj], bf16_lo(w.x), o[hl][0]);
-                        o[hl][1] = fmaf(pj[jj], bf16_hi(w.x), o[hl][1]);
-                        o[hl][CPL > 2 ? 2 : 0] = fmaf(pj[jj], bf16_lo(w.y), o[hl][CPL > 2 ? 2 : 0]);
-                        o[hl][CPL > 3 ? 3 : 0] = fmaf(pj[jj], bf16_hi(w.y), o[hl][CPL > 3 ? 3 : 0]);
+        for (int ks = 0; ks < MBW; ++ks) {
+            uint32_t bh[NCT][2], bl[NCT][2];
+#pragma unroll
+            for (int ct = 0; ct < NCT; ++ct) {
+                const bool hv_ok = head_ok(ct, gq);
+                const uint32_t off = static_cast<uint32_t>((head_of(ct, hv_ok ? gq : 0) * PS + ks * 16 + 2 * tq) * 2);
+                uint32_t h0 = 0u, h1 = 0u, l0 = 0u, l1 = 0u;
+                if (hv_ok) {
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(h0) : "r"(pb_hi_a + off));
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(h1) : "r"(pb_hi_a + off + 16));
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(l0) : "r"(pb_lo_a + off));
+                    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(l1) : "r"(pb_lo_a + off + 16));
+                }
+                bh[ct][0] = h0;
+                bh[ct][1] = h1;
+                bl[ct][0] = l0;
+                bl[ct][1] = l1;
+            }
+            const int pos = mb0 * 16 + ks * 16 + ld_pos;  // position row (in the tile) of this lane
+            // this thread's A elements cover positions ks*16 + 2tq (+1, +8, +9) of the slice
+            const int pa = ks * 16 + 2 * tq;
+            const bool ragged = lim < ROWS;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int dim = mt * 16 + ld_dim;
+                const int dh = dim >> 6, chunk = (dim & 63) >> 3;
+                uint32_t a0 = 0u, a1 = 0u, a2 = 0u, a3 = 0u;
+#pragma unroll
+                for (int ct = 0; ct < NCT; ++ct) {
+                    if (ct == 0 || VPK == 2) {
+                        const uint32_t addr = sbase + kStageBytes +
+                                              static_cast<uint32_t>((vh_ct[ct] * DH + dh) * g.P * 128 + pos * 128 +
+                                                                    ((chunk ^ (pos & 7)) << 4));
+                        ldmatrix_x4_trans(addr, a0, a1, a2, a3);
+                        if (ragged) {
+                            // positions past l: zero the value elements so that
+                            // whatever the cache holds there cannot reach the sum
+                            const uint32_t m0 = (pa < lim ? 0xffffu : 0u) | (pa + 1 < lim ? 0xffff0000u : 0u);
+                            const uint32_t m8 = (pa + 8 < lim ? 0xffffu : 0u) | (pa + 9 < lim ? 0xffff0000u : 0u);
+                            a0 &= m0;
+                            a1 &= m0;
+                            a2 &= m8;
+                            a3 &= m8;
+                        }
                     }
+                    mma_16816(o[mt][ct], a0, a1, a2, a3, bh[ct][0], bh[ct][1]);
+                    mma_16816(o[mt][ct], a0, a1, a2, a3, bl[ct][0], bl[ct][1]);
                 }
             }
         }
@@ -258,11 +322,11 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     if (!ok && lane == 0) raise_device_error(a.err, kErrTimeout);
 }
 
-template <int D, int NT>
+template <int D, int NT, int NCT>
 cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, const DenseArgs& a,
                      cudaStream_t stream) {
     const size_t smem = dense_smem_bytes(a.g, a.stages);
-    auto kern = dense_kernel<D, NT>;
+    auto kern = dense_kernel<D, NT, NCT>;
     static const cudaError_t attr = cudaFuncSetAttribute(
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem);
     if (attr != cudaSuccess) return attr;
@@ -273,6 +337,11 @@ cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, const Den
 
 }  // namespace
 
+bool dense_supported(const Geometry& g) {
+    // each key head's query heads use one value head, or two whole ones
+    return g.hv <= 2 * g.hk && (g.hv % g.hk == 0 || g.hk % g.hv == 0);
+}
+
 size_t dense_stage_bytes(const Geometry& g) {
     return static_cast<size_t>(kStageBytes) + static_cast<size_t>(g.P) * g.hv * g.d * 2;
 }
@@ -280,16 +349,21 @@ size_t dense_stage_bytes(const Geometry& g) {
 size_t dense_smem_bytes(const Geometry& g, int stages) {
     const size_t hs = static_cast<size_t>(g.NT) * 8;
     return 1024 + stages * dense_stage_bytes(g) +
-           kConsumerWarps * hs * (kPStride + 1) * sizeof(float) + 2 * stages * sizeof(uint64_t) + 16;
+           kConsumerWarps * hs * (2 * weight_stride(g.d) * sizeof(uint16_t) + sizeof(float)) +
+           2 * stages * sizeof(uint64_t) + 16;
 }
 
 cudaError_t launch_dense(const CUtensorMap& kmap, const CUtensorMap& vmap, const DenseArgs& a,
                          cudaStream_t stream) {
+    if (!dense_supported(a.g)) return cudaErrorInvalidValue;
     const int d = a.g.d, nt = a.g.NT;
-    if (d == 64 && nt == 1) return launch_t<64, 1>(kmap, vmap, a, stream);
-    if (d == 64 && nt == 2) return launch_t<64, 2>(kmap, vmap, a, stream);
-    if (d == 128 && nt == 1) return launch_t<128, 1>(kmap, vmap, a, stream);
-    if (d == 128 && nt == 2) return launch_t<128, 2>(kmap, vmap, a, stream);
+    const bool two = a.g.hv > a.g.hk || nt == 2;  // two column tiles of query heads
+    if (d == 64 && nt == 1) return two ? launch_t<64, 1, 2>(kmap, vmap, a, stream)
+                                       : launch_t<64, 1, 1>(kmap, vmap, a, stream);
+    if (d == 64 && nt == 2) return launch_t<64, 2, 2>(kmap, vmap, a, stream);
+    if (d == 128 && nt == 1) return two ? launch_t<128, 1, 2>(kmap, vmap, a, stream)
+                                        : launch_t<128, 1, 1>(kmap, vmap, a, stream);
+    if (d == 128 && nt == 2) return launch_t<128, 2, 2>(kmap, vmap, a, stream);
     return cudaErrorInvalidValue;
 }
 

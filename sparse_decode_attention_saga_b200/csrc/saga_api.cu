@@ -416,7 +416,7 @@ int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const
     Geometry g;
     int st = make_geometry(dims, &g);
     if (st) return st;
-    if (g.hv > 2 * g.hk) return SAGA_ERR_UNSUPPORTED;
+    if (!dense_supported(g)) return SAGA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !out || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
         !aligned(out, 4))
         return SAGA_ERR_INVALID_ARG;
@@ -432,7 +432,7 @@ int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const
 
     CUtensorMap kmap, vmap;
     if ((st = encode_cache_map(&kmap, k, g, g.hk, true))) return st;
-    if ((st = encode_cache_map(&vmap, v, g, g.hv, false))) return st;
+    if ((st = encode_cache_map(&vmap, v, g, g.hv, true))) return st;
     DenseArgs a{};
     a.g = g;
     a.C = stream_ctas(g, dev, 1);

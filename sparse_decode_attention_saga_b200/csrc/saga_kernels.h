@@ -120,6 +120,9 @@ struct DenseArgs {
     float* records;
     uint32_t* err;
 };
+// Shapes the dense kernel handles: h_v <= 2 h_k, value heads aligned with
+// the key-head groups.
+bool dense_supported(const Geometry& g);
 size_t dense_stage_bytes(const Geometry& g);
 size_t dense_smem_bytes(const Geometry& g, int stages);
 cudaError_t launch_dense(const CUtensorMap& kmap, const CUtensorMap& vmap, const DenseArgs& a,
