@@ -1,192 +1,16 @@
-// Log-sum-exp merge of the partial records of one (batch, query head) row,
-// and the empty-set fallback.
-//
-// Each partial record holds (m, l, count, m_all, o[d]) with
-// o = sum_j exp(s_j - m) V_j and l = sum_j exp(s_j - m) over the part's kept
-// entries.  The merge is M = max m_r, out = sum_r exp(m_r - M) o_r /
-// sum_r exp(m_r - M) l_r (split-K / flash-decoding combine).
-//
-// Empty-set reading (the pages are silent): when a stale threshold lies above
-// every logit of the row, nothing was kept and the row keeps its maximal
-// entries instead (tau_eff = min(tau, max_j s_j)).  The streaming kernel
-// recorded the maximum logit each part saw; here the row's logits are
-// recomputed with the same tensor-core routine (bit-identical values), the
-// positions equal to that maximum are found, and their value rows averaged
-// (equal logits give equal softmax weights).
-#include "qk_tile.cuh"
-#include "saga_kernels.h"
+// The combine kernel: one CTA per (batch, query head) row merges the row's
+// partial records (combine_row.cuh).  Used after the dense kernel; the
+// sparse paths merge in the gather kernel's last CTA of each row.
+#include "combine_row.cuh"
 
 namespace saga {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
-
 template <int D, int NT>
-__device__ void fallback_row(const CombineArgs& a, long long row, float m_star, float* out_row,
-                             int32_t* cnt_out, uint8_t* kbuf) {
-    const Geometry& g = a.g;
-    const int lane = threadIdx.x & 31;
-    const int bb = static_cast<int>(row / g.hq);
-    const int i = static_cast<int>(row - static_cast<long long>(bb) * g.hq);
-    const int kh = i / g.G, hl = i - kh * g.G;
-    const int vh = i * g.hv / g.hq;
-    const int nti = hl >> 3, col = hl & 7;
-    const int gq = lane >> 2, tq = lane & 3;
-    constexpr int DH = D / 64;
-    constexpr int CPL = D / 32;  // value columns per lane
-
-    QFrag<D, NT> qf;
-    load_q_frag<D, NT>(qf, reinterpret_cast<const __nv_bfloat16*>(a.q), g.hq, g.G, bb, kh, lane);
-    const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(a.k);
-    const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(a.v);
-    float osum[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) osum[c] = 0.f;
-    int count = 0;
-    for (int j0 = 0; j0 < g.l; j0 += 16) {
-        // 16 key rows of head kh into the swizzled tile layout of qk_mma
-        for (int q8 = lane; q8 < 16 * D / 8; q8 += 32) {
-            const int r = q8 / (D / 8), cc = q8 - r * (D / 8);
-            const int dh = cc >> 3, c8 = cc & 7;
-            const int pos = j0 + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (pos < g.l)
-                v = *reinterpret_cast<const uint4*>(
-                    K + ((static_cast<size_t>(bb) * g.l_cap + pos) * g.hk + kh) * D + cc * 8);
-            *reinterpret_cast<uint4*>(kbuf + dh * 16 * 128 + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
-        }
-        __syncwarp();
-        float acc[1][NT][4];
-        qk_mma<D, NT, 1>(smem_addr(kbuf), 16, 0, 0, qf, acc, lane);
-        __syncwarp();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            bool match = false;
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float s = __fmul_rn(acc[0][nt][2 * h + e], g.scale);
-                    const int pos = j0 + gq + 8 * h;
-                    if (nt == nti && 2 * tq + e == col && pos < g.l && s == m_star) match = true;
-                }
-            uint32_t ball = __ballot_sync(0xffffffffu, match);
-            while (ball) {
-                const int src = __ffs(ball) - 1;
-                ball &= ball - 1;
-                const int pos = j0 + (src >> 2) + 8 * h;
-                const __nv_bfloat16* vr =
-                    V + ((static_cast<size_t>(bb) * g.l_cap + pos) * g.hv + vh) * D + lane * CPL;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) osum[c] += __bfloat162float(vr[c]);
-                ++count;
-            }
-        }
-    }
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) out_row[lane * CPL + c] = osum[c] / static_cast<float>(count);
-    if (lane == 0 && cnt_out) *cnt_out = count;
-    (void)DH;
-}
-
-template <int D, int NT>
-__global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a) {
-    __shared__ float red[3][kWarps];
-    __shared__ int red_c[kWarps];
-    __shared__ float red_o[kWarps][D];
-    __shared__ __align__(1024) uint8_t kbuf[16 * D * 2];
-
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const CombineArgs a) {
     pdl_wait();  // the partial records come from the previous kernel
-    const Geometry& g = a.g;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const long long row = blockIdx.x;
-    const int bb = static_cast<int>(row / g.hq);
-    int R;
-    if (a.mode == kCombineParts) {
-        R = a.parts;
-    } else {
-        const long long T = static_cast<long long>(g.b) * g.tiles;
-        R = slots_of_batch(bb, g.tiles, T, a.C) * a.recs_per_slot;
-    }
-    const float* recs = a.records + static_cast<size_t>(row) * g.S_cap * g.WPK * g.rec;
-
-    float M = -kInf, mall = -kInf;
-    int cnt = 0;
-    for (int r = tid; r < R; r += kThreads) {
-        const float* rec = recs + static_cast<size_t>(r) * g.rec;
-        M = fmaxf(M, rec[0]);
-        mall = fmaxf(mall, rec[3]);
-        cnt += __float_as_int(rec[2]);
-    }
-    M = warp_max(M);
-    mall = warp_max(mall);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-    if (lane == 0) {
-        red[0][warp] = M;
-        red[1][warp] = mall;
-        red_c[warp] = cnt;
-    }
-    __syncthreads();
-    M = red[0][0];
-    mall = red[1][0];
-    cnt = red_c[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) {
-        M = fmaxf(M, red[0][w]);
-        mall = fmaxf(mall, red[1][w]);
-        cnt += red_c[w];
-    }
-
-    float* out_row = a.out + static_cast<size_t>(row) * D;
-    if (cnt == 0 && a.fallback) {
-        if (warp == 0) fallback_row<D, NT>(a, row, mall, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf);
-        return;
-    }
-
-    float lsum = 0.f;
-    for (int r = tid; r < R; r += kThreads) {
-        const float* rec = recs + static_cast<size_t>(r) * g.rec;
-        const float m = rec[0];
-        if (m > -kInf) lsum += rec[1] * __expf(m - M);
-    }
-    lsum = warp_sum(lsum);
-    __syncthreads();
-    if (lane == 0) red[2][warp] = lsum;
-    __syncthreads();
-    lsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) lsum += red[2][w];
-    const float inv = 1.f / lsum;
-
-    // Records are spread over the warps (warp w sums records w, w+4, ...;
-    // lane owns D/32 columns), so the loads of different records are in
-    // flight together; the warps' partial sums are then added in a fixed order.
-    constexpr int CPL = D / 32;
-    float o[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) o[c] = 0.f;
-    for (int r = warp; r < R; r += kWarps) {
-        const float* rec = recs + static_cast<size_t>(r) * g.rec;
-        const float m = rec[0];
-        if (m > -kInf) {
-            const float wgt = __expf(m - M);
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) o[c] = fmaf(rec[kRecHeader + lane * CPL + c], wgt, o[c]);
-        }
-    }
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) red_o[warp][lane * CPL + c] = o[c];
-    __syncthreads();
-    for (int c = tid; c < D; c += kThreads) {
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) v += red_o[w][c];
-        out_row[c] = v * inv;
-    }
-    if (tid == 0 && a.sel_cnt) a.sel_cnt[row] = cnt;
+    combine_row<D, NT>(a, blockIdx.x);
 }
 
 }  // namespace
@@ -194,7 +18,7 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const CombineArgs a) 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream) {
     const unsigned rows = static_cast<unsigned>(static_cast<long long>(a.g.b) * a.g.hq);
     const int d = a.g.d, nt = a.g.NT;
-    const dim3 grid(rows), block(kThreads);
+    const dim3 grid(rows), block(kCombineThreads);
     if (d == 64 && nt == 1) return launch_dependent(combine_kernel<64, 1>, grid, block, 0, stream, a);
     if (d == 64 && nt == 2) return launch_dependent(combine_kernel<64, 2>, grid, block, 0, stream, a);
     if (d == 128 && nt == 1) return launch_dependent(combine_kernel<128, 1>, grid, block, 0, stream, a);

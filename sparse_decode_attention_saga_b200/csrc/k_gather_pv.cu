@@ -21,8 +21,7 @@
 // (tau_eff <= max), so no running max is needed.  The share's (m, sum of
 // weights, count, row max, unnormalised output) record is merged across
 // shares by the combine kernel.
-#include "saga_device.cuh"
-#include "saga_kernels.h"
+#include "combine_row.cuh"
 
 namespace saga {
 
@@ -42,7 +41,9 @@ constexpr int kMinShare = 128;  // kept entries per CTA at least
 constexpr int kGatherInflight = SAGA_GATHER_INFLIGHT;
 constexpr int kGatherMinBlocks = SAGA_GATHER_MINBLOCKS;
 
-template <int D>
+static_assert(kThreads == kCombineThreads, "the last CTA of a row runs the row merge");
+
+template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(const GatherArgs a) {
     constexpr int LPR = D * 2 / 16;    // lanes per value row (16 B each)
     constexpr int RPI = 32 / LPR;      // value rows per warp instruction
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     __shared__ float red_o[kWarps][D];
     __shared__ int red_i[kWarps];
     __shared__ long long row_base;
+    __shared__ int is_last;
 
     pdl_wait();     // lists, counts and maxima come from the previous kernel
     pdl_trigger();
@@ -259,6 +261,16 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
         rec[2] = __int_as_float(n);
         rec[3] = m_all;
     }
+
+    // the row's last CTA to finish merges the row's records
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) is_last = atomicAdd(a.tickets + row, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!is_last) return;
+    __threadfence();
+    if (tid == 0) a.tickets[row] = 0u;
+    combine_row<D, NT>(a.cmb, row);
 }
 
 }  // namespace
@@ -270,18 +282,20 @@ size_t gather_smem_bytes(int max_lists, int max_slots) {
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
     const dim3 grid(a.parts, static_cast<unsigned>(static_cast<long long>(a.g.b) * a.g.hq));
     const size_t smem = gather_smem_bytes(a.max_lists, a.max_slots);
-    if (smem > static_cast<size_t>(kGatherMaxSmem)) return cudaErrorInvalidValue;
-    if (a.g.d == 64) {
-        static const cudaError_t attr = cudaFuncSetAttribute(
-            gather_pv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem);
-        if (attr != cudaSuccess) return attr;
-        return launch_dependent(gather_pv_kernel<64>, grid, dim3(kThreads), smem, stream, a);
-    } else {
-        static const cudaError_t attr = cudaFuncSetAttribute(
-            gather_pv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem);
-        if (attr != cudaSuccess) return attr;
-        return launch_dependent(gather_pv_kernel<128>, grid, dim3(kThreads), smem, stream, a);
+    if (smem > static_cast<size_t>(kGatherMaxSmem) || a.cmb.parts != a.parts) return cudaErrorInvalidValue;
+#define SAGA_GATHER_CASE(D_, NT_)                                                                  \
+    if (a.g.d == D_ && a.g.NT == NT_) {                                                            \
+        static const cudaError_t attr = cudaFuncSetAttribute(                                     \
+            gather_pv_kernel<D_, NT_>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem); \
+        if (attr != cudaSuccess) return attr;                                                      \
+        return launch_dependent(gather_pv_kernel<D_, NT_>, grid, dim3(kThreads), smem, stream, a); \
     }
+    SAGA_GATHER_CASE(64, 1)
+    SAGA_GATHER_CASE(64, 2)
+    SAGA_GATHER_CASE(128, 1)
+    SAGA_GATHER_CASE(128, 2)
+#undef SAGA_GATHER_CASE
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace saga

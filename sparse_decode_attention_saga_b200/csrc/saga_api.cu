@@ -344,19 +344,15 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         ga.cnt = sa.cnt;
         ga.rowmax = sa.rowmax;
         ga.records = records;
-        e = launch_gather_pv(ga, s);
+        ga.tickets = ws_at<uint32_t>(ws, L.tickets);
+        ga.cmb.g = g;
+        ga.cmb.mode = kCombineParts;
+        ga.cmb.parts = ga.parts;
+        ga.cmb.records = records;
+        ga.cmb.out = out;
+        ga.cmb.sel_cnt = sel_cnt;
         g_launches += 1;
-        if (e != cudaSuccess) return SAGA_ERR_CUDA;
-
-        CombineArgs ca{};
-        ca.g = g;
-        ca.mode = kCombineParts;
-        ca.parts = ga.parts;
-        ca.records = records;
-        ca.out = out;
-        ca.sel_cnt = sel_cnt;
-        g_launches += 1;
-        return cuda_status(launch_combine(ca, s));
+        return cuda_status(launch_gather_pv(ga, s));
     }
 
     // fused: stream K, compare on chip, lists -> gathered PV -> combine
@@ -392,23 +388,19 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     ga.seg_cnt = a.seg_cnt;
     ga.seg_mall = a.seg_mall;
     ga.records = records;
-    e = launch_gather_pv(ga, s);
+    ga.tickets = ws_at<uint32_t>(ws, L.tickets);
+    ga.cmb.g = g;
+    ga.cmb.mode = kCombineParts;
+    ga.cmb.parts = ga.parts;
+    ga.cmb.fallback = 1;
+    ga.cmb.q = q;
+    ga.cmb.k = k;
+    ga.cmb.v = v;
+    ga.cmb.records = records;
+    ga.cmb.out = out;
+    ga.cmb.sel_cnt = sel_cnt;
     g_launches += 1;
-    if (e != cudaSuccess) return SAGA_ERR_CUDA;
-
-    CombineArgs ca{};
-    ca.g = g;
-    ca.mode = kCombineParts;
-    ca.parts = ga.parts;
-    ca.fallback = 1;
-    ca.q = q;
-    ca.k = k;
-    ca.v = v;
-    ca.records = records;
-    ca.out = out;
-    ca.sel_cnt = sel_cnt;
-    g_launches += 1;
-    return cuda_status(launch_combine(ca, s));
+    return cuda_status(launch_gather_pv(ga, s));
 }
 
 int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const void* v,

@@ -86,6 +86,25 @@ struct SelectArgs {
 };
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream);
 
+// Log-sum-exp merge of partial records, plus the empty-set fallback.
+enum CombineMode : int {
+    kCombineParts = 0,     // `parts` records per row (gathered contiguous lists)
+    kCombineSlots = 1,     // slots_of_batch records per row (fused / dense kernels)
+};
+struct CombineArgs {
+    Geometry g;
+    int mode;
+    int parts;
+    int C;
+    int recs_per_slot;  // kCombineSlots: 1 (gathered lists) or WPK (dense kernel)
+    int fallback;  // recompute logits from q/K for rows that kept nothing
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* records;
+    float* out;
+    int32_t* sel_cnt;
+};
 // Gathered softmax-PV over kept lists -> partial records.
 enum ListMode : int {
     kListContiguous = 0,  // idx [rows][l], cnt [rows], s from logits
@@ -107,6 +126,10 @@ struct GatherArgs {
     const int32_t* seg_cnt;
     const float* seg_mall;
     float* records;
+    // The last CTA of each row (per-row tickets, zero on entry and left at
+    // zero) merges the row's `parts` records as cmb describes.
+    uint32_t* tickets;
+    CombineArgs cmb;
 };
 size_t gather_smem_bytes(int max_lists, int max_slots);
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream);
@@ -128,25 +151,6 @@ size_t dense_smem_bytes(const Geometry& g, int stages);
 cudaError_t launch_dense(const CUtensorMap& kmap, const CUtensorMap& vmap, const DenseArgs& a,
                          cudaStream_t stream);
 
-// Log-sum-exp merge of partial records, plus the empty-set fallback.
-enum CombineMode : int {
-    kCombineParts = 0,     // `parts` records per row (gathered contiguous lists)
-    kCombineSlots = 1,     // slots_of_batch records per row (fused / dense kernels)
-};
-struct CombineArgs {
-    Geometry g;
-    int mode;
-    int parts;
-    int C;
-    int recs_per_slot;  // kCombineSlots: 1 (gathered lists) or WPK (dense kernel)
-    int fallback;  // recompute logits from q/K for rows that kept nothing
-    const void* q;
-    const void* k;
-    const void* v;
-    const float* records;
-    float* out;
-    int32_t* sel_cnt;
-};
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 
 }  // namespace saga
