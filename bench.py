@@ -423,7 +423,7 @@ def run_ours(args, world, rank, local):
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "bytes_per_launch": kern_bytes, "us_per_launch": kern_us,
                      "traffic": measured_traffic(w.name)},
-        "step_roofline": {"what": "reuse step (fused kernel + gather + combine) vs ideal bytes "
+        "step_roofline": {"what": "reuse step (streaming kernel + gather with row merge) vs ideal bytes "
                                   "K + distinct kept V rows + q/tau/out",
                           "ideal_bytes": step_ideal, "us": us_reuse,
                           "achieved": step_ideal / (us_reuse * 1e-6) / 1e9,
