@@ -400,6 +400,29 @@ def run_ours(args, world, rank, local):
     barrier(world)
     e2e_us = max_over_ranks(e0.elapsed_time(e1) * 1e3 / args.steps, world)
 
+    # ---- decode with cache growth: each step appends its own K/V rows and attends
+    # over l + 1 positions.  The cache memory is reused: the decoder starts at
+    # l_kv - G and re-appends rows l_kv - G .. l_kv - 1 (the same values).
+    G = 32
+    rows_k = K[:, w.l_kv - G:w.l_kv].transpose(0, 1).contiguous()   # [G, b, h_k, d]
+    rows_v = V[:, w.l_kv - G:w.l_kv].transpose(0, 1).contiguous()
+    grow_us = []
+    for rep in range(2):  # the first pass warms up
+        gdec = AtopNDecoder(w.batch, w.h_q, w.h_k, w.h_v, w.head_dim, w.l_kv - G, w.N, w.n,
+                            l_cap=w.l_kv)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g0.record(stream)
+            for t in range(G):
+                gdec.append(rows_k[t], rows_v[t], K, V)
+                gdec.step(t, qs[t % qs.shape[0]], K, V)
+            g1.record(stream)
+        stream.synchronize()
+        assert gdec.error() == _lib.SAGA_OK
+        grow_us.append(g0.elapsed_time(g1) * 1e3 / G)
+        del gdec
+    del rows_k, rows_v
+
     line = {
         "metric": METRIC, "value": us_per_step, "unit": "us/step", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": us_per_step / 1e3,
@@ -428,6 +451,9 @@ def run_ours(args, world, rank, local):
                           "ideal_bytes": step_ideal, "us": us_reuse,
                           "achieved": step_ideal / (us_reuse * 1e-6) / 1e9,
                           "frac": step_ideal / (us_reuse * 1e-6) / 1e9 / peak},
+        "grow": {"us_per_step": grow_us[-1], "steps": G, "l_kv": [w.l_kv - G + 1, w.l_kv],
+                 "what": "append this step's K/V rows, then the Atop-N step over the grown "
+                         "cache (refresh every n), eager, CUDA events"},
         "e2e": {"value": e2e_us, "unit": "us/step",
                 "h2d_bytes_per_step": int(qs[0].numel() * 2),
                 "d2h_bytes_per_step": int(dec.out.numel() * 4)},

@@ -29,7 +29,8 @@
  *
  * Supported shapes: head_dim in {64, 128}; h_k in {1, 2, 4, 8}; h_q a
  * multiple of h_k and of h_v with h_q/h_k <= 16 and h_q <= 128;
- * saga_decode_dense also needs h_v <= 2*h_k; 1 <= l_kv <= l_cap;
+ * saga_decode_dense also needs h_v <= 2*h_k with h_v a multiple or a
+ * divisor of h_k; 1 <= l_kv <= l_cap;
  * batch*l_cap < 2^31.  Others return SAGA_ERR_UNSUPPORTED.
  *
  * Conventions shared by every call:
@@ -45,6 +46,8 @@
  *     error nothing is launched and no output is touched.
  *   - Workspace: `ws` must hold saga_workspace_bytes(dims, N) bytes and must
  *     be zeroed once after allocation (or passed to saga_workspace_reset).
+ *     A workspace sized for dims with a larger l_kv (all else equal) serves
+ *     every shorter length, so a growing cache needs one sized for l_cap.
  *     Calls that share a workspace must be ordered on one stream.
  *   - Device-side faults: kernels bound every wait; a wait that runs out
  *     sets a sticky flag in the workspace that saga_workspace_error reads.
@@ -153,6 +156,20 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
  * SAGA_ERR_WORKSPACE (too many rows), SAGA_ERR_DEVICE, SAGA_ERR_CUDA. */
 int saga_topn_refresh_noalloc(const saga_dims* dims, int32_t N, const float* logits_in,
                               float* thresh_out, saga_stream_t stream);
+
+/* Cache growth (real decode: each generated token appends its own key and
+ * value rows before it attends; "More Value per Key" measures latency over
+ * 32 generated tokens, ai.info summary, Main Findings).  Writes
+ *   k_new [batch, h_k, head_dim] bf16 -> k[b, l_kv, :, :]
+ *   v_new [batch, h_v, head_dim] bf16 -> v[b, l_kv, :, :]
+ * i.e. at the first free row of each batch element's cache; the caller then
+ * decodes with l_kv + 1.  The thresholds of the last refresh stay valid for
+ * the grown cache (the new position is compared like any other).
+ * Errors: SAGA_ERR_INVALID_ARG (l_kv >= l_cap: no free row; null or
+ * misaligned pointer; bad dims), SAGA_ERR_UNSUPPORTED, SAGA_ERR_DEVICE,
+ * SAGA_ERR_CUDA. */
+int saga_cache_append(const saga_dims* dims, const void* k_new, const void* v_new, void* k,
+                      void* v, saga_stream_t stream);
 
 /* Failure-path self-test (the paper has no counterpart): one CTA waits, with
  * the bounded wait every pipelined kernel uses, on a barrier that nothing

@@ -27,7 +27,7 @@ EXPORTS = (
     "saga_workspace_bytes", "saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
     "saga_workspace_reset", "saga_workspace_error", "saga_status_string", "saga_launch_count",
     "saga_set_kernel_events", "saga_version", "saga_topn_refresh_noalloc",
-    "saga_selftest_wait_timeout",
+    "saga_selftest_wait_timeout", "saga_cache_append",
 )
 
 
@@ -67,6 +67,8 @@ def load(path: str | None = None):
         lib.saga_atopn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, SZ, P]
         lib.saga_topn_refresh_noalloc.argtypes = [D, I32, P, P, P]
         lib.saga_topn_refresh_noalloc.restype = ctypes.c_int
+        lib.saga_cache_append.argtypes = [D, P, P, P, P, P]
+        lib.saga_cache_append.restype = ctypes.c_int
         lib.saga_selftest_wait_timeout.argtypes = [P, SZ, ctypes.c_uint32, P]
         lib.saga_selftest_wait_timeout.restype = ctypes.c_int
         lib.saga_workspace_reset.argtypes = [P, SZ, P]
@@ -142,6 +144,13 @@ def topn_refresh_noalloc(d, N, logits_in, thresh_out, stream=None) -> None:
     st = load().saga_topn_refresh_noalloc(ctypes.byref(d), int(N), _ptr(logits_in),
                                           _ptr(thresh_out), _stream(stream))
     _check("saga_topn_refresh_noalloc", st)
+
+
+def cache_append(d, k_new, v_new, k, v, stream=None) -> None:
+    """Write this step's new key/value rows at position d.l_kv of the caches."""
+    _check("saga_cache_append",
+           load().saga_cache_append(ctypes.byref(d), _ptr(k_new), _ptr(v_new), _ptr(k), _ptr(v),
+                                    _stream(stream)))
 
 
 def selftest_wait_timeout(ws, limit_us: int, stream=None) -> None:

@@ -449,6 +449,32 @@ int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const
     return cuda_status(launch_combine(ca, s));
 }
 
+int saga_cache_append(const saga_dims* dims, const void* k_new, const void* v_new, void* k,
+                      void* v, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (g.l >= g.l_cap) return SAGA_ERR_INVALID_ARG;  // no room for the new row
+    if (!k_new || !v_new || !k || !v || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+        !aligned(k, 16) || !aligned(v, 16))
+        return SAGA_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    AppendArgs a{};
+    a.b = g.b;
+    a.hk = g.hk;
+    a.hv = g.hv;
+    a.d = g.d;
+    a.l_cap = g.l_cap;
+    a.pos = g.l;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.k = k;
+    a.v = v;
+    g_launches += 1;
+    return cuda_status(launch_cache_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int saga_workspace_reset(void* ws, size_t ws_bytes, saga_stream_t stream) {
     if (!ws) return SAGA_ERR_INVALID_ARG;
     return cuda_status(cudaMemsetAsync(ws, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream)));

@@ -153,4 +153,15 @@ cudaError_t launch_dense(const CUtensorMap& kmap, const CUtensorMap& vmap, const
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 
+// Cache growth: new rows k_new [b,h_k,d], v_new [b,h_v,d] -> row `pos` of
+// k [b,l_cap,h_k,d] and v [b,l_cap,h_v,d].
+struct AppendArgs {
+    int b, hk, hv, d, l_cap, pos;
+    const void* k_new;
+    const void* v_new;
+    void* k;
+    void* v;
+};
+cudaError_t launch_cache_append(const AppendArgs& a, cudaStream_t stream);
+
 }  // namespace saga

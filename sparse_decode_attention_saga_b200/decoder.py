@@ -15,17 +15,41 @@ from . import _lib
 
 
 class AtopNDecoder:
+    """Decode-loop state for one layer.  The cache holds l_kv valid rows out of
+    l_cap; ``append`` adds the step's own key/value rows (the cached length
+    grows by one), so buffers are sized for l_cap."""
+
     def __init__(self, batch, h_q, h_k, h_v, head_dim, l_kv, N, n, l_cap=None, device="cuda"):
-        self.dims = _lib.dims(batch, h_q, h_k, h_v, head_dim, l_kv, l_cap)
+        self.l_cap = int(l_kv if l_cap is None else l_cap)
+        self.dims = _lib.dims(batch, h_q, h_k, h_v, head_dim, l_kv, self.l_cap)
         self.N, self.n = int(N), int(n)
         self.device = torch.device(device)
-        nbytes = _lib.workspace_bytes(self.dims, self.N)
+        # a workspace sized for the full capacity serves every shorter length
+        nbytes = _lib.workspace_bytes(_lib.dims(batch, h_q, h_k, h_v, head_dim, self.l_cap,
+                                                self.l_cap), self.N)
         if nbytes == 0:
             raise _lib.SagaError("saga_workspace_bytes", _lib.SAGA_ERR_UNSUPPORTED)
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
         self.thresh = torch.full((batch, h_q), float("nan"), dtype=torch.float32, device=self.device)
-        self.logits = torch.empty((batch, h_q, l_kv), dtype=torch.float32, device=self.device)
+        self._logits = torch.empty(batch * h_q * self.l_cap, dtype=torch.float32, device=self.device)
         self.out = torch.empty((batch, h_q, head_dim), dtype=torch.float32, device=self.device)
+
+    @property
+    def l_kv(self) -> int:
+        return int(self.dims.l_kv)
+
+    @property
+    def logits(self) -> torch.Tensor:
+        """[b, h_q, l_kv] view of the logits buffer (written on refresh steps)."""
+        d = self.dims
+        return self._logits[: d.batch * d.h_q * d.l_kv].view(d.batch, d.h_q, d.l_kv)
+
+    def append(self, k_new, v_new, k, v, stream=None) -> None:
+        """Writes this step's key/value rows ([b,h_k,d], [b,h_v,d] bf16) at
+        position l_kv of the caches; the following steps see l_kv + 1 rows."""
+        _lib.cache_append(self.dims, k_new, v_new, k, v, stream)
+        d = self.dims
+        self.dims = _lib.dims(d.batch, d.h_q, d.h_k, d.h_v, d.head_dim, d.l_kv + 1, self.l_cap)
 
     @classmethod
     def for_workload(cls, w, device="cuda"):

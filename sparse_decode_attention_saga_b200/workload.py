@@ -129,6 +129,23 @@ def make_queries(w: Workload, seed: int = 0, device="cpu", steps: int | None = N
     return (z + base).to(torch.bfloat16)
 
 
+def make_new_rows(w: Workload, seed: int = 0, device="cpu", steps: int | None = None):
+    """Key and value rows generated one per decode step, for a growing cache:
+    ([steps, b, h_k, d], [steps, b, h_v, d]) bf16, drawn like the cache rows
+    (N(0,1); each (step, batch, key head) key row gets 2*u_k added with
+    probability 2 %)."""
+    steps = w.steps if steps is None else steps
+    u = topic_vectors(w, seed, device)
+    g = _gen(seed * 7919 + 4, device)
+    kf = torch.randn(steps, w.batch, w.h_k, w.head_dim, generator=g, device=device,
+                     dtype=torch.float32)
+    shift = torch.rand(steps, w.batch, w.h_k, generator=g, device=device) < TOPIC_FRACTION
+    kf += TOPIC_SHIFT * shift[..., None].float() * u[None, None]
+    vf = torch.randn(steps, w.batch, w.h_v, w.head_dim, generator=g, device=device,
+                     dtype=torch.float32)
+    return kf.to(torch.bfloat16), vf.to(torch.bfloat16)
+
+
 def bf16_bits(t: torch.Tensor):
     """A bf16 tensor as a numpy uint16 array of its bit patterns (host copy)."""
     assert t.dtype == torch.bfloat16
