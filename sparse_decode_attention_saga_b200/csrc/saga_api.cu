@@ -355,12 +355,16 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         return cuda_status(launch_gather_pv(ga, s));
     }
 
-    // fused: stream K, compare on chip, lists -> gathered PV -> combine
+    // fused: stream K, compare on chip, lists -> gathered PV with the row merge
+    const int C = stream_ctas(g, dev);
+    const int slots = max_slots(g, static_cast<long long>(g.b) * g.tiles, C);
+    if (gather_smem_bytes(slots * g.WPK, slots) > static_cast<size_t>(kGatherMaxSmem))
+        return SAGA_ERR_UNSUPPORTED;  // checked before anything is enqueued
     CUtensorMap kmap;
     if ((st = encode_cache_map(&kmap, k, g, g.hk, true))) return st;
     StreamArgs a{};
     a.g = g;
-    a.C = stream_ctas(g, dev);
+    a.C = C;
     a.stages = kStreamStages;
     a.q = q;
     a.thresh = thresh;
@@ -379,10 +383,8 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     ga.mode = kListSegments;
     ga.C = a.C;
     ga.parts = gather_parts(g, dev);
-    ga.max_slots = max_slots(g, static_cast<long long>(g.b) * g.tiles, a.C);
-    ga.max_lists = ga.max_slots * g.WPK;
-    if (gather_smem_bytes(ga.max_lists, ga.max_slots) > static_cast<size_t>(kGatherMaxSmem))
-        return SAGA_ERR_UNSUPPORTED;
+    ga.max_slots = slots;
+    ga.max_lists = slots * g.WPK;
     ga.v = v;
     ga.seg_list = a.list;
     ga.seg_cnt = a.seg_cnt;
