@@ -21,16 +21,30 @@ using namespace saga;
 
 namespace {
 
-// Pipeline depth and CTAs per SM of the streaming kernels (tuning constants):
-// 3 x 32 KB of K per CTA, two CTAs per SM.
-#ifndef SAGA_STREAM_STAGES
-#define SAGA_STREAM_STAGES 3
+// Ring shape of the streaming kernels (tuning constants, measured on B200):
+// with head_dim 64 and one n-tile of query heads per key head (G <= 8) one
+// CTA per SM with a 6 x 32 KB ring of K streams best; with more tensor-core
+// and compare work per byte (two n-tiles, or head_dim 128) two CTAs per SM
+// with 3 x 32 KB each hide it better.
+#ifndef SAGA_STREAM_STAGES_NT1
+#define SAGA_STREAM_STAGES_NT1 6
 #endif
-#ifndef SAGA_STREAM_CTAS_PER_SM
-#define SAGA_STREAM_CTAS_PER_SM 2
+#ifndef SAGA_STREAM_CTAS_PER_SM_NT1
+#define SAGA_STREAM_CTAS_PER_SM_NT1 1
 #endif
-constexpr int kStreamStages = SAGA_STREAM_STAGES;
-constexpr int kStreamCtasPerSm = SAGA_STREAM_CTAS_PER_SM;
+#ifndef SAGA_STREAM_STAGES_NT2
+#define SAGA_STREAM_STAGES_NT2 3
+#endif
+#ifndef SAGA_STREAM_CTAS_PER_SM_NT2
+#define SAGA_STREAM_CTAS_PER_SM_NT2 2
+#endif
+struct StreamShape {
+    int stages, ctas_per_sm;
+};
+StreamShape stream_shape(const Geometry& g) {
+    return g.NT == 1 && g.d == 64 ? StreamShape{SAGA_STREAM_STAGES_NT1, SAGA_STREAM_CTAS_PER_SM_NT1}
+                     : StreamShape{SAGA_STREAM_STAGES_NT2, SAGA_STREAM_CTAS_PER_SM_NT2};
+}
 constexpr long long kMinTilesPerCta = 4;
 constexpr int kMaxDevices = 64;
 
@@ -150,7 +164,7 @@ int max_slots(const Geometry& g, long long T, int C) {
 
 // Grid of the streaming kernels: `per_sm` CTAs per SM, at most one per tile, and
 // never more partial-record slots per batch row than the workspace holds.
-int stream_ctas(const Geometry& g, const DeviceInfo& dev, int per_sm = kStreamCtasPerSm) {
+int stream_ctas(const Geometry& g, const DeviceInfo& dev, int per_sm) {
     const long long T = static_cast<long long>(g.b) * g.tiles;
     long long c = static_cast<long long>(dev.sms) * per_sm;
     if (c > kMaxCtas) c = kMaxCtas;
@@ -216,8 +230,8 @@ int run_logits(const Geometry& g, const DeviceInfo& dev, const void* q, const vo
     if (st) return st;
     StreamArgs a{};
     a.g = g;
-    a.C = stream_ctas(g, dev);
-    a.stages = kStreamStages;
+    a.C = stream_ctas(g, dev, stream_shape(g).ctas_per_sm);
+    a.stages = stream_shape(g).stages;
     a.q = q;
     a.logits = dst;
     a.err = err;
@@ -356,7 +370,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     }
 
     // fused: stream K, compare on chip, lists -> gathered PV with the row merge
-    const int C = stream_ctas(g, dev);
+    const int C = stream_ctas(g, dev, stream_shape(g).ctas_per_sm);
     const int slots = max_slots(g, static_cast<long long>(g.b) * g.tiles, C);
     if (gather_smem_bytes(slots * g.WPK, slots) > static_cast<size_t>(kGatherMaxSmem))
         return SAGA_ERR_UNSUPPORTED;  // checked before anything is enqueued
@@ -365,7 +379,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     StreamArgs a{};
     a.g = g;
     a.C = C;
-    a.stages = kStreamStages;
+    a.stages = stream_shape(g).stages;
     a.q = q;
     a.thresh = thresh;
     a.list = ws_at<int2>(ws, L.list_idx);  // spans the list_idx and list_s regions
