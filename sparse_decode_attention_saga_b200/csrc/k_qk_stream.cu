@@ -79,6 +79,9 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
         // ---------------------------------------------------------- producer
         if (lane == 0) {
             prefetch_tensor_map(&kmap);
+            // K is read once per step: its lines go first, so that the kept
+            // lists and logits written meanwhile stay in L2 for the next kernel
+            const uint64_t k_policy = l2_policy_evict_first();
             int issued = 0;
             int bb = static_cast<int>(t0 / g.tiles);
             int tl = static_cast<int>(t0 - static_cast<long long>(bb) * g.tiles);
@@ -91,8 +94,8 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
                 uint8_t* dst = smem + static_cast<size_t>(st) * kStageBytes;
                 for (int kh = 0; kh < g.hk; ++kh)
                     for (int dh = 0; dh < DH; ++dh)
-                        tma_load_3d(dst + (kh * DH + dh) * g.P * 128, &kmap, &full[st], dh * 64,
-                                    kh, z);
+                        tma_load_3d_hint(dst + (kh * DH + dh) * g.P * 128, &kmap, &full[st],
+                                         dh * 64, kh, z, k_policy);
                 issued = k + 1;
                 if (++tl == g.tiles) {
                     tl = 0;
