@@ -47,7 +47,6 @@ template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(const GatherArgs a) {
     constexpr int LPR = D * 2 / 16;    // lanes per value row (16 B each)
     constexpr int RPI = 32 / LPR;      // value rows per warp instruction
-    constexpr int UNROLL = 8;
     constexpr int MBW = 128 / D;
 
     extern __shared__ int table[];     // pre, start, slot_pos, slot_len

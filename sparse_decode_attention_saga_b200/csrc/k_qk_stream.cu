@@ -153,24 +153,26 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
     };
 
     auto end_segment = [&](int bb) {
-        if (MODE != kStreamSelect) return;
+        if constexpr (MODE == kStreamSelect) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float m = mall[nt][e];  // raw accumulator max; scaling is monotone
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-                m = __fmul_rn(m, scale);
-                const int hl = nt * 8 + 2 * tq + e;
-                if (gq == 0 && hl < G) {
-                    const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + hl;
-                    const size_t at = (row * g.S_cap + slot) * g.WPK + sub;
-                    a.seg_cnt[at] = cnt[nt][e];
-                    a.seg_mall[at] = m;
+                for (int e = 0; e < 2; ++e) {
+                    float m = mall[nt][e];  // raw accumulator max; scaling is monotone
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+                    m = __fmul_rn(m, scale);
+                    const int hl = nt * 8 + 2 * tq + e;
+                    if (gq == 0 && hl < G) {
+                        const size_t row = static_cast<size_t>(bb) * g.hq + kh * G + hl;
+                        const size_t at = (row * g.S_cap + slot) * g.WPK + sub;
+                        a.seg_cnt[at] = cnt[nt][e];
+                        a.seg_mall[at] = m;
+                    }
                 }
-            }
+        }
+        (void)bb;
     };
 
     // Tile epilogue: logits store, or compare + list append, for the tile

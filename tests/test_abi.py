@@ -127,3 +127,17 @@ def test_missing_library_fails_loudly(tmp_path):
             _lib.load(missing)
     finally:
         _lib.load(_lib.LIBRARY)
+
+
+def test_cache_append_validation(lib):
+    full = _lib.dims(1, 4, 1, 2, 64, 64, 64)        # l_kv == l_cap: no free row
+    assert lib.saga_cache_append(ctypes.byref(full), 16, 16, 16, 16, None) == \
+        _lib.SAGA_ERR_INVALID_ARG
+    d = _lib.dims(1, 4, 1, 2, 64, 64, 65)
+    assert lib.saga_cache_append(ctypes.byref(d), None, 16, 16, 16, None) == \
+        _lib.SAGA_ERR_INVALID_ARG                   # null new key row
+    assert lib.saga_cache_append(ctypes.byref(d), 16, 16, 24, 16, None) == \
+        _lib.SAGA_ERR_INVALID_ARG                   # misaligned key cache
+    bad = _lib.dims(1, 4, 1, 2, 96, 64, 65)
+    assert lib.saga_cache_append(ctypes.byref(bad), 16, 16, 16, 16, None) == \
+        _lib.SAGA_ERR_UNSUPPORTED
