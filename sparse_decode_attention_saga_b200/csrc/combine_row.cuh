@@ -91,11 +91,22 @@ __device__ void fallback_row(const CombineArgs& a, long long row, float m_star, 
     (void)DH;
 }
 
-// Merges row `row`'s records into out (all kCombineThreads threads of the
-// block take part; it contains block barriers).  Records are read through
-// L2, so a CTA of the kernel that wrote them may merge them.
+// Number of partial records of row (of batch element bb).
+__device__ __forceinline__ int row_records(const CombineArgs& a, int bb) {
+    if (a.mode == kCombineParts) return a.parts;
+    const Geometry& g = a.g;
+    const long long T = static_cast<long long>(g.b) * g.tiles;
+    return slots_of_batch(bb, g.tiles, T, a.C) * a.recs_per_slot;
+}
+
+// Merges records r_begin .. r_begin + R - 1 of row `row` (R < 0: all the
+// row's records) into out, or, with partial_out, into one partial record
+// (m, l, count, m_all, o) without normalising.  All kCombineThreads threads
+// of the block take part (block barriers).  Records are read through L2, so
+// a CTA of the kernel that wrote them may merge them.
 template <int D, int NT>
-__device__ void combine_row(const CombineArgs& a, long long row) {
+__device__ void combine_row(const CombineArgs& a, long long row, int r_begin = 0, int R = -1,
+                            float* partial_out = nullptr) {
     constexpr int kWarps = kCombineThreads / 32;
     constexpr int kThreads = kCombineThreads;
     __shared__ float red[3][kWarps];
@@ -106,14 +117,9 @@ __device__ void combine_row(const CombineArgs& a, long long row) {
     const Geometry& g = a.g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int bb = static_cast<int>(row / g.hq);
-    int R;
-    if (a.mode == kCombineParts) {
-        R = a.parts;
-    } else {
-        const long long T = static_cast<long long>(g.b) * g.tiles;
-        R = slots_of_batch(bb, g.tiles, T, a.C) * a.recs_per_slot;
-    }
-    const float* recs = a.records + static_cast<size_t>(row) * g.S_cap * g.WPK * g.rec;
+    if (R < 0) R = row_records(a, bb);
+    const float* recs =
+        a.records + (static_cast<size_t>(row) * g.S_cap * g.WPK + r_begin) * g.rec;
 
     float M = -kInf, mall = -kInf;
     int cnt = 0;
@@ -144,7 +150,7 @@ __device__ void combine_row(const CombineArgs& a, long long row) {
     }
 
     float* out_row = a.out + static_cast<size_t>(row) * D;
-    if (cnt == 0 && a.fallback) {
+    if (cnt == 0 && a.fallback && !partial_out) {
         if (warp == 0)
             fallback_row<D, NT>(a, row, mall, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf);
         return;
@@ -163,34 +169,56 @@ __device__ void combine_row(const CombineArgs& a, long long row) {
     lsum = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) lsum += red[2][w];
-    const float inv = 1.f / lsum;
+    const float inv = partial_out ? 1.f : 1.f / lsum;
 
-    // Records are spread over the warps (warp w sums records w, w+4, ...;
+    // Records are spread over the warps (warp w sums records w, w+8, ...;
     // lane owns D/32 columns), so the loads of different records are in
     // flight together; the warps' partial sums are then added in a fixed order.
     constexpr int CPL = D / 32;
     float o[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) o[c] = 0.f;
-    for (int r = warp; r < R; r += kWarps) {
-        const float* rec = recs + static_cast<size_t>(r) * g.rec;
-        const float m = __ldcg(rec);
-        if (m > -kInf) {
-            const float wgt = __expf(m - M);
+    // eight records per warp in flight: their loads are issued before any is used
+    constexpr int U = 8;
+    for (int r0 = warp; r0 < R; r0 += U * kWarps) {
+        float mv[U], ov[U][CPL];
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) o[c] = fmaf(__ldcg(rec + kRecHeader + lane * CPL + c), wgt, o[c]);
+        for (int u = 0; u < U; ++u) {
+            const int r = r0 + u * kWarps;
+            const float* rec = recs + static_cast<size_t>(r < R ? r : 0) * g.rec;
+            mv[u] = r < R ? __ldcg(rec) : -kInf;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) ov[u][c] = __ldcg(rec + kRecHeader + lane * CPL + c);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (mv[u] > -kInf) {
+                const float wgt = __expf(mv[u] - M);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) o[c] = fmaf(ov[u][c], wgt, o[c]);
+            }
         }
     }
 #pragma unroll
     for (int c = 0; c < CPL; ++c) red_o[warp][lane * CPL + c] = o[c];
     __syncthreads();
+    float* dst = partial_out ? partial_out + kRecHeader : out_row;
     for (int c = tid; c < D; c += kThreads) {
         float v = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) v += red_o[w][c];
-        out_row[c] = v * inv;
+        dst[c] = v * inv;
     }
-    if (tid == 0 && a.sel_cnt) a.sel_cnt[row] = cnt;
+    if (tid == 0) {
+        if (partial_out) {
+            partial_out[0] = M;
+            partial_out[1] = lsum;
+            partial_out[2] = __int_as_float(cnt);
+            partial_out[3] = mall;
+        } else if (a.sel_cnt) {
+            a.sel_cnt[row] = cnt;
+        }
+    }
 }
 
 }  // namespace saga

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -47,6 +48,7 @@ StreamShape stream_shape(const Geometry& g) {
 }
 constexpr long long kMinTilesPerCta = 4;
 constexpr int kMaxDevices = 64;
+constexpr long long kMaxGatherParts = 32;
 
 std::atomic<uint64_t> g_launches{0};
 thread_local cudaEvent_t t_ev_start = nullptr;
@@ -185,6 +187,9 @@ int gather_parts(const Geometry& g, const DeviceInfo& dev) {
     long long parts = (8ll * dev.sms + rows - 1) / rows;
     const long long cap = static_cast<long long>(g.S_cap) * g.WPK;
     if (parts > cap) parts = cap;
+    // few rows: each part still wants >= 128 kept entries, so more parts than
+    // this only add CTAs that build the list table and exit
+    if (parts > kMaxGatherParts) parts = kMaxGatherParts;
     return static_cast<int>(parts < 1 ? 1 : parts);
 }
 
@@ -461,6 +466,15 @@ int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const
     ca.recs_per_slot = g.WPK;
     ca.records = a.records;
     ca.out = out;
+    // Many records per row (few rows, many slots): several CTAs per row merge
+    // shares of about 64 records into partial records stored past the inputs.
+    const int r_max = max_slots(g, static_cast<long long>(g.b) * g.tiles, a.C) * g.WPK;
+    const int chunks = r_max > 128 ? std::min(32, (r_max + 63) / 64) : 1;
+    if (chunks > 1 && r_max + chunks <= g.S_cap * g.WPK) {
+        ca.chunks = chunks;
+        ca.partial_slot = r_max;
+        ca.tickets = ws_at<uint32_t>(ws, L.tickets);
+    }
     g_launches += 1;
     return cuda_status(launch_combine(ca, s));
 }

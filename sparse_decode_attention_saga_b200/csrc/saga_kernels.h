@@ -97,7 +97,10 @@ struct CombineArgs {
     int parts;
     int C;
     int recs_per_slot;  // kCombineSlots: 1 (gathered lists) or WPK (dense kernel)
-    int fallback;  // recompute logits from q/K for rows that kept nothing
+    int chunks;        // CTAs per row (0 or 1: one CTA merges the row)
+    int partial_slot;  // chunks > 1: record slot of chunk 0's partial (past the inputs)
+    uint32_t* tickets; // chunks > 1: per-row tickets, zero on entry and left at zero
+    int fallback;      // recompute logits from q/K for rows that kept nothing
     const void* q;
     const void* k;
     const void* v;
