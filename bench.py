@@ -345,6 +345,21 @@ def run_ours(args, world, rank, local):
     us_dense = time_steps(lambda r: dec.dense(qs[r % 4], K, V, out=dense_out), 10)
     us_mix = (us_refresh + (w.n - 1) * us_reuse) / w.n
 
+    # Dense grouped-query attention of the layer SAGA was converted from
+    # (h_k = h_v): the pages' full-attention baseline.  Its own cache (more
+    # key heads) is drawn with the same recipe.
+    if w.h_k != w.h_v:
+        wg = w.scaled(h_k=w.h_v)
+        Kg, Vg = make_cache(wg, seed, "cuda")
+        gdec = AtopNDecoder.for_workload(wg)
+        gqa_out = torch.empty_like(gdec.out)
+        us_dense_gqa = time_steps(lambda r: gdec.dense(qs[r % 4], Kg, Vg, out=gqa_out), 10)
+        assert gdec.error() == _lib.SAGA_OK
+        del Kg, Vg, gdec, gqa_out
+        torch.cuda.empty_cache()
+    else:
+        us_dense_gqa = us_dense
+
     # ---- dominant kernel: the fused compare kernel of the reuse step
     kern_us = []
     ks, ke = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -440,6 +455,8 @@ def run_ours(args, world, rank, local):
         "us_reuse_step": us_reuse, "us_refresh_step": us_refresh,
         "us_mean_step_1_in_n": us_mix,
         "us_dense_step": us_dense, "speedup_vs_dense": us_dense / us_per_step,
+        "us_dense_gqa_step": us_dense_gqa, "speedup_vs_dense_gqa": us_dense_gqa / us_per_step,
+        "dense_gqa": f"h_k = h_v = {w.h_v} (the GQA layer before key-head merging)",
         "kept_entries_per_step": kept, "distinct_value_rows": U,
         "roofline": {"kernel": "qk_stream_kernel (fused compare, reuse step)", "bound": "hbm",
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
