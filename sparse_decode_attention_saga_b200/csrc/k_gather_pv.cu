@@ -173,14 +173,25 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     constexpr int INFLIGHT = ROUNDS < kGatherInflight ? ROUNDS : kGatherInflight;
 
     // entry e -> (position, logit); out-of-range entries give (0, -inf)
+    // The list holding entry e is the last j with pre[j] <= e.  Each lane's
+    // entries only move forward (by 32 per round); with d = 64 a cursor `lo`
+    // stays put while the entry is still inside its list (one compare) and
+    // otherwise moves by binary search over the later lists; with d = 128 the
+    // extra live register costs more than it saves (measured), so every
+    // lookup is a binary search.
+    int lo = 0;
     auto fetch = [&](int e, int& pos, float& s) {
         pos = 0;
         s = -kInf;
         if (e < w1) {
-            int lo = 0, hi = nl - 1;  // last list j with pre[j] <= e
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (pre[mid] <= e) lo = mid; else hi = mid - 1;
+            if (D != 64) lo = 0;
+            if (lo + 1 < nl && pre[lo + 1] <= e) {
+                int l2 = lo + 1, hi = nl - 1;
+                while (l2 < hi) {
+                    const int mid = (l2 + hi + 1) >> 1;
+                    if (pre[mid] <= e) l2 = mid; else hi = mid - 1;
+                }
+                lo = l2;
             }
             const long long at = row_base + start[lo] + (e - pre[lo]);
             if (a.mode == kListContiguous) {
