@@ -13,7 +13,10 @@
 // and takes a ticket; the CTA that takes the last ticket scans the histogram
 // from the top bin, fixes the digit that holds the rank, and stores
 // (prefix, rank) for the next pass, or the threshold after the last pass.
-// No CTA waits for another.
+// No CTA waits for another.  With a candidate buffer, pass 1 also copies the
+// logits of its prefix bucket into its chunk's part of the buffer (one
+// shared-memory counter per CTA, reserved a warp at a time), and pass 2 reads
+// only those candidates, each CTA its own chunk's.
 #include "saga_device.cuh"
 #include "saga_kernels.h"
 
@@ -47,8 +50,10 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t& e
     return total;
 }
 
+// Eight CTAs per SM on the vectorised path: the grid sizing (radix_chunks)
+// counts on them (the scalar path keeps its registers).
 template <int PASS, int VEC>
-__global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a) {
+__global__ void __launch_bounds__(kThreads, VEC == 4 ? 8 : 4) radix_pass_kernel(const RadixArgs a) {
     constexpr int kLoadsV = kLoads / VEC;  // VEC-wide loads per thread per round
     constexpr int shift = PASS == 0 ? 21 : (PASS == 1 ? 10 : 0);
     constexpr int width = PASS == 2 ? 10 : 11;
@@ -59,6 +64,7 @@ __global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a)
     __shared__ uint32_t hist[nb];
     __shared__ uint32_t warp_tot[kThreads / 32];
     __shared__ int is_last;
+    __shared__ int s_cand;  // pass 1: candidates this CTA has copied out
 
     pdl_wait();  // logits, histograms and the previous pass's state
     pdl_trigger();
@@ -66,13 +72,17 @@ __global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a)
     const long long row = blockIdx.y;
     const int chunk = blockIdx.x;
     for (int i = tid; i < nb; i += kThreads) hist[i] = 0;
+    if (tid == 0) s_cand = 0;
     const uint32_t prefix = PASS == 0 ? 0u : __ldcg(a.state + row * 2);
     __syncthreads();
+    const int lane = tid & 31;
+    const bool from_cand = PASS == 2 && a.cand != nullptr;
 
     const float* src = a.logits + row * a.l;
     const int per = ((a.l + a.chunks - 1) / a.chunks + 3) & ~3;  // multiple of 4
-    const int j0 = chunk * per;
-    const int j1 = min(a.l, j0 + per);
+    const int j0 = from_cand ? 0 : chunk * per;
+    const int j1 = from_cand ? 0 : min(a.l, j0 + per);
+    float* cdst = PASS == 1 && a.cand ? a.cand + row * a.l + static_cast<long long>(chunk) * per : nullptr;
     // 64 bytes of independent coalesced loads per thread per round (16-byte
     // loads when the rows are 16-byte aligned) keep enough bytes in flight to
     // stream the logits at HBM speed.
@@ -91,6 +101,7 @@ __global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a)
                 for (int c = 0; c < VEC; ++c) v[k][c] = j + c < j1 ? __ldg(src + j + c) : 0.f;
             }
         }
+        uint32_t cm = 0u;  // pass 1: which of this round's values are bucket members
 #pragma unroll
         for (int k = 0; k < kLoadsV; ++k) {
 #pragma unroll
@@ -99,17 +110,51 @@ __global__ void __launch_bounds__(kThreads) radix_pass_kernel(const RadixArgs a)
                 const uint32_t key = float_to_key(v[k][c]);
                 const bool cand = j < j1 && (PASS == 0 || (key >> high) == prefix);
                 if (cand) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+                if (PASS == 1 && cand) cm |= 1u << (k * VEC + c);
+            }
+        }
+        if (PASS == 1 && cdst) {
+            // copy this round's bucket members out: a warp-wide scan of the
+            // per-thread counts, one shared-memory reservation per warp
+            const int mine = __popc(cm);
+            int inc = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += x;
+            }
+            const int wtot = __shfl_sync(0xffffffffu, inc, 31);
+            if (wtot > 0) {
+                int wbase = 0;
+                if (lane == 31) wbase = atomicAdd(&s_cand, wtot);
+                wbase = __shfl_sync(0xffffffffu, wbase, 31);
+                int at = wbase + inc - mine;
+#pragma unroll
+                for (int k = 0; k < kLoadsV; ++k)
+#pragma unroll
+                    for (int c = 0; c < VEC; ++c)
+                        if (cm & (1u << (k * VEC + c))) cdst[at++] = v[k][c];
             }
         }
     }
+    if (from_cand) {
+        // pass 2 over the candidates pass 1 copied out of this chunk
+        const int n = min(max(__ldcg(a.cand_cnt + row * kRadixMaxChunks + chunk), 0), per);
+        const float* cs = a.cand + row * a.l + static_cast<long long>(chunk) * per;
+        for (int j = tid; j < n; j += kThreads) {
+            const uint32_t key = float_to_key(__ldcg(cs + j));
+            if ((key >> high) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+        }
+    }
     __syncthreads();
+    if (PASS == 1 && cdst && tid == 0) a.cand_cnt[row * kRadixMaxChunks + chunk] = s_cand;
 
     uint32_t* ghist = a.hist + (static_cast<long long>(PASS) * a.rows + row) * kRadixBins;
     for (int i = tid; i < nb; i += kThreads)
         if (hist[i]) atomicAdd(ghist + i, hist[i]);
     __threadfence();
     __syncthreads();
-    if (tid == 0) is_last = (atomicAdd(a.tickets + row, 1u) == static_cast<uint32_t>(a.chunks - 1));
+    if (tid == 0) is_last = (atomicAdd(a.tickets + row, 1u) == gridDim.x - 1);
     __syncthreads();
     if (!is_last) return;
     __threadfence();

@@ -204,7 +204,7 @@ int radix_chunks(long long rows, int l, int sms) {
     const long long max_chunks = (l + 4095) / 4096;
     long long best = 1;
     double best_cost = 1e300;
-    for (long long c = 1; c <= max_chunks && c <= 64; ++c) {
+    for (long long c = 1; c <= max_chunks && c <= kRadixMaxChunks; ++c) {
         const long long waves = (rows * c + slots - 1) / slots;
         const double cost = static_cast<double>(waves) * (static_cast<double>((l + c - 1) / c) + 3000.0);
         if (cost < best_cost) {
@@ -305,6 +305,10 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
     r.tickets = ws_at<uint32_t>(ws, L.tickets);
     r.thresh = thresh_out;
     r.err = err;
+    // pass 1 copies its bucket's logits into the kept-list region (unused
+    // until the decode call) so that pass 2 reads only those
+    r.cand = ws_at<float>(ws, L.list_idx);
+    r.cand_cnt = ws_at<int32_t>(ws, L.cand_cnt);
     g_launches += kRadixPasses;
     return cuda_status(launch_radix_select(r, s));
 }

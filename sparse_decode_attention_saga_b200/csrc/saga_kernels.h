@@ -65,6 +65,12 @@ struct RadixArgs {
     uint32_t* tickets;
     float* thresh;
     uint32_t* err;
+    // Optional (nullable): pass 1 also copies the logits of its prefix bucket
+    // into chunk c's part [c*per, c*per + per) of cand[row][0..l) and their
+    // number into cand_cnt[row][c]; pass 2 then reads only those (chunk c's
+    // CTA its own chunk's).  Null: pass 2 reads the whole row again.
+    float* cand;
+    int32_t* cand_cnt;
 };
 cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream);
 // CTAs per row for the radix passes (cost model over waves and per-CTA overhead).

@@ -32,6 +32,8 @@ constexpr uint32_t kErrTimeout = 1u;
 // Radix select: 32-bit keys in digits of 11, 11 and 10 bits.
 constexpr int kRadixBins = 2048;
 constexpr int kRadixPasses = 3;
+// CTAs per row of a radix pass at most (sizes the candidate counts).
+constexpr int kRadixMaxChunks = 64;
 // Partial record: m (kept max), l (sum of exp), count, m_all, o[d].
 constexpr int kRecHeader = 4;
 
@@ -69,6 +71,7 @@ struct WsLayout {
     size_t state;     // uint32 [b*hq][2]  (prefix, rank)
     size_t tickets;   // uint32 [b*hq]
     size_t cnt;       // int32  [b*hq]
+    size_t cand_cnt;  // int32  [b*hq][kRadixMaxChunks]  radix pass-1 candidates per chunk
     size_t rowmax;    // float  [b*hq]
     size_t seg_cnt;   // int32  [b*hq][S_cap][WPK]
     size_t seg_mall;  // float  [b*hq][S_cap][WPK]
@@ -95,6 +98,7 @@ inline WsLayout workspace_layout(const Geometry& g) {
     w.state = take(rows * 2 * sizeof(uint32_t));
     w.tickets = take(rows * sizeof(uint32_t));
     w.cnt = take(rows * sizeof(int32_t));
+    w.cand_cnt = take(rows * kRadixMaxChunks * sizeof(int32_t));
     w.rowmax = take(rows * sizeof(float));
     w.seg_cnt = take(rows * g.S_cap * g.WPK * sizeof(int32_t));
     w.seg_mall = take(rows * g.S_cap * g.WPK * sizeof(float));
