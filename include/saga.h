@@ -15,22 +15,26 @@
  * Shapes and layouts (all row-major, innermost last; bf16 = IEEE bfloat16):
  *   q      [batch, h_q, head_dim]            bf16   this step's queries
  *   k      [batch, l_cap, h_k, head_dim]     bf16   key cache
- *   v      [batch, l_cap, h_v, head_dim]     bf16   value cache
+ *   v      [batch, l_cap, h_v, v_head_dim]   bf16   value cache
  *          positions 0 .. l_kv-1 of each batch element are valid; rows
  *          l_kv .. l_cap-1 are capacity and are never used.
  *   logits [batch, h_q, l_kv]                fp32   s = q.k / sqrt(head_dim)
  *   thresh [batch, h_q]                      fp32   Atop-N thresholds (tau)
- *   out    [batch, h_q, head_dim]            fp32
+ *   out    [batch, h_q, v_head_dim]          fp32
  *   sel_idx[batch, h_q, l_kv]                int32  kept positions, ascending,
  *                                                   first sel_cnt entries valid
  *   sel_cnt[batch, h_q]                      int32
  * Head maps: query head i reads key head i*h_k/h_q and value head i*h_v/h_q
  * (contiguous groups, as in grouped-query attention).
  *
- * Supported shapes: head_dim in {64, 128}; h_k in {1, 2, 4, 8}; h_q a
+ * Supported shapes: head_dim = v_head_dim in {64, 128}, or head_dim 32 with
+ * v_head_dim 64 and h_k >= 2 (keys of half the value dim: the pages' Sigma-
+ * style head layout, Main Findings "Head count beats head dimension");
+ * h_k in {1, 2, 4, 8}; h_q a
  * multiple of h_k and of h_v with h_q/h_k <= 16 and h_q <= 128;
  * saga_decode_dense also needs h_v <= 2*h_k with h_v a multiple or a
- * divisor of h_k; 1 <= l_kv <= l_cap;
+ * divisor of h_k, and a stage (32 KB of keys and the value rows of the
+ * same positions) that fits twice in shared memory; 1 <= l_kv <= l_cap;
  * batch*l_cap < 2^31.  Others return SAGA_ERR_UNSUPPORTED.
  *
  * Conventions shared by every call:
@@ -71,9 +75,10 @@ typedef struct {
     int32_t h_q;       /* query heads                          */
     int32_t h_k;       /* key heads   (SAGA: h_k < h_v allowed) */
     int32_t h_v;       /* value heads                          */
-    int32_t head_dim;  /* d, shared by keys and values         */
+    int32_t head_dim;  /* d_k: key (and query) head dim        */
     int32_t l_kv;      /* valid cached positions               */
     int32_t l_cap;     /* cache capacity (row stride in positions) */
+    int32_t v_head_dim; /* d_v: value head dim; 0 means d_k    */
 } saga_dims;
 
 typedef enum {
@@ -161,7 +166,7 @@ int saga_topn_refresh_noalloc(const saga_dims* dims, int32_t N, const float* log
  * value rows before it attends; "More Value per Key" measures latency over
  * 32 generated tokens, ai.info summary, Main Findings).  Writes
  *   k_new [batch, h_k, head_dim] bf16 -> k[b, l_kv, :, :]
- *   v_new [batch, h_v, head_dim] bf16 -> v[b, l_kv, :, :]
+ *   v_new [batch, h_v, v_head_dim] bf16 -> v[b, l_kv, :, :]
  * i.e. at the first free row of each batch element's cache; the caller then
  * decodes with l_kv + 1.  The thresholds of the last refresh stay valid for
  * the grown cache (the new position is compared like any other).

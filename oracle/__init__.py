@@ -11,7 +11,9 @@ in ``oracle.cpp`` next to this file, with the readings of the pages it takes.
 
 Arrays: bf16 tensors travel as ``numpy.uint16`` bit patterns, logits and
 outputs as ``float32``.  Shapes: q [b,hq,d], K [b,l_cap,hk,d],
-V [b,l_cap,hv,d], logits [b,hq,l], tau [b,hq], out [b,hq,d].
+V [b,l_cap,hv,dv], logits [b,hq,l], tau [b,hq], out [b,hq,dv] (dv = d except
+for the Sigma-style layout with narrower keys, Main Findings "Head count
+beats head dimension").
 """
 from __future__ import annotations
 
@@ -66,8 +68,8 @@ class Oracle:
         lib.oracle_nth_largest_sort.argtypes = [P, L, L, L, P]
         lib.oracle_select.argtypes = [P, L, L, P, P, P]
         lib.oracle_attend_masked.argtypes = [L] * 6 + [P, P, P, P]
-        lib.oracle_decode_dense.argtypes = [L] * 7 + [P, P, P, P]
-        lib.oracle_atopn_step.argtypes = [L] * 10 + [P] * 8
+        lib.oracle_decode_dense.argtypes = [L] * 8 + [P, P, P, P]
+        lib.oracle_atopn_step.argtypes = [L] * 11 + [P] * 8
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         for f in (lib.oracle_logits, lib.oracle_nth_largest, lib.oracle_nth_largest_sort,
@@ -141,12 +143,13 @@ class Oracle:
     def decode_dense(self, q, K, V, l: int | None = None) -> np.ndarray:
         """Full attention over the first ``l`` cached positions."""
         q, K, V = _u16(q), _u16(K), _u16(V)
-        b, hq, d = q.shape
+        b, hq, dk = q.shape
         _, l_cap, hk, _ = K.shape
-        hv = V.shape[2]
+        hv, dv = V.shape[2], V.shape[3]
         l = l_cap if l is None else l
-        out = np.empty((b, hq, d), np.float32)
-        rc = self.lib.oracle_decode_dense(b, hq, hk, hv, d, l, l_cap, _p(q), _p(K), _p(V), _p(out))
+        out = np.empty((b, hq, dv), np.float32)
+        rc = self.lib.oracle_decode_dense(b, hq, hk, hv, dk, dv, l, l_cap, _p(q), _p(K), _p(V),
+                                          _p(out))
         assert rc == 0
         return out
 
@@ -155,17 +158,17 @@ class Oracle:
         """One Atop-N decode step; ``tau_state`` [b,hq] float32 is updated in
         place on refresh steps (t mod n == 0).  Returns (out, logits, mask, cnt)."""
         q, K, V = _u16(q), _u16(K), _u16(V)
-        b, hq, d = q.shape
+        b, hq, dk = q.shape
         _, l_cap, hk, _ = K.shape
-        hv = V.shape[2]
+        hv, dv = V.shape[2], V.shape[3]
         l = l_cap if l is None else l
         assert tau_state.dtype == np.float32 and tau_state.shape == (b, hq)
         assert tau_state.flags["C_CONTIGUOUS"]
-        out = np.empty((b, hq, d), np.float32)
+        out = np.empty((b, hq, dv), np.float32)
         s = np.empty((b, hq, l), np.float32)
         mask = np.empty((b, hq, l), np.uint8)
         cnt = np.empty((b, hq), np.int32)
-        rc = self.lib.oracle_atopn_step(b, hq, hk, hv, d, l, l_cap, N, t, n,
+        rc = self.lib.oracle_atopn_step(b, hq, hk, hv, dk, dv, l, l_cap, N, t, n,
                                         _p(q), _p(K), _p(V), _p(tau_state), _p(out),
                                         _p(s), _p(mask), _p(cnt))
         assert rc == 0

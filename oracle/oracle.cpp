@@ -10,7 +10,9 @@
 // Contributions", "Main Findings", "Methodology in Plain English") and on
 // atlas.scime.ai (sections "Approach", "Experimental setup").
 //
-// Notation: b batch, hq/hk/hv query/key/value heads, d head dim, l cached
+// Notation: b batch, hq/hk/hv query/key/value heads, d head dim (dk for keys
+// and queries, dv for values where they differ: the Sigma-style head layout
+// of Main Findings, "Head count beats head dimension"), l cached
 // positions (first l rows of a cache with capacity l_cap), N top-N budget,
 // n refresh interval, t 0-based decode step.
 //
@@ -212,14 +214,15 @@ int oracle_attend_masked(long b, long hq, long hv, long d, long l, long l_cap,
 
 // Full (dense) attention, the speedup denominator (Main Findings, "end-to-end
 // decoding speedups ... over baseline full attention"): every position kept.
-int oracle_decode_dense(long b, long hq, long hk, long hv, long d, long l, long l_cap,
+// dk: key/query head dim (logits), dv: value head dim (output).
+int oracle_decode_dense(long b, long hq, long hk, long hv, long dk, long dv, long l, long l_cap,
                         const uint16_t* q, const uint16_t* K, const uint16_t* V,
                         float* out) {
     if (l <= 0) return -1;
     std::vector<float> s(static_cast<size_t>(b * hq * l));
-    if (oracle_logits(b, hq, hk, d, l, l_cap, q, K, s.data()) != 0) return -1;
+    if (oracle_logits(b, hq, hk, dk, l, l_cap, q, K, s.data()) != 0) return -1;
     std::vector<uint8_t> mask(s.size(), 1);
-    return oracle_attend_masked(b, hq, hv, d, l, l_cap, s.data(), mask.data(), V, out);
+    return oracle_attend_masked(b, hq, hv, dv, l, l_cap, s.data(), mask.data(), V, out);
 }
 
 // One Atop-N decode step in the order the method states it (Key
@@ -228,7 +231,7 @@ int oracle_decode_dense(long b, long hq, long hk, long hv, long d, long l, long 
 // softmax over the kept entries; gathered value sum.
 // tau_state [b,hq] is read and, on refresh steps, overwritten.
 // s_out [b,hq,l] and mask_out [b,hq,l] / cnt_out [b,hq] are optional.
-int oracle_atopn_step(long b, long hq, long hk, long hv, long d, long l, long l_cap,
+int oracle_atopn_step(long b, long hq, long hk, long hv, long dk, long dv, long l, long l_cap,
                       long N, long t, long n,
                       const uint16_t* q, const uint16_t* K, const uint16_t* V,
                       float* tau_state, float* out, float* s_out,
@@ -236,12 +239,12 @@ int oracle_atopn_step(long b, long hq, long hk, long hv, long d, long l, long l_
     if (l <= 0 || N <= 0 || n <= 0 || t < 0) return -1;
     const long rows = b * hq;
     std::vector<float> s(static_cast<size_t>(rows * l));
-    if (oracle_logits(b, hq, hk, d, l, l_cap, q, K, s.data()) != 0) return -1;
+    if (oracle_logits(b, hq, hk, dk, l, l_cap, q, K, s.data()) != 0) return -1;
     if (t % n == 0) oracle_nth_largest(s.data(), rows, l, N, tau_state);
     std::vector<uint8_t> mask(s.size());
     std::vector<int32_t> cnt(static_cast<size_t>(rows));
     oracle_select(s.data(), rows, l, tau_state, mask.data(), cnt.data());
-    const int rc = oracle_attend_masked(b, hq, hv, d, l, l_cap, s.data(), mask.data(), V, out);
+    const int rc = oracle_attend_masked(b, hq, hv, dv, l, l_cap, s.data(), mask.data(), V, out);
     if (s_out) std::copy(s.begin(), s.end(), s_out);
     if (mask_out) std::copy(mask.begin(), mask.end(), mask_out);
     if (cnt_out) std::copy(cnt.begin(), cnt.end(), cnt_out);

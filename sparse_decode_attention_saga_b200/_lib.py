@@ -34,7 +34,7 @@ EXPORTS = (
 class SagaDims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_k", ctypes.c_int32),
                 ("h_v", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("l_kv", ctypes.c_int32),
-                ("l_cap", ctypes.c_int32)]
+                ("l_cap", ctypes.c_int32), ("v_head_dim", ctypes.c_int32)]
 
 
 class SagaError(RuntimeError):
@@ -106,8 +106,11 @@ def _check(fn: str, status: int) -> None:
         raise SagaError(fn, status)
 
 
-def dims(batch, h_q, h_k, h_v, head_dim, l_kv, l_cap=None) -> SagaDims:
-    return SagaDims(batch, h_q, h_k, h_v, head_dim, l_kv, l_kv if l_cap is None else l_cap)
+def dims(batch, h_q, h_k, h_v, head_dim, l_kv, l_cap=None, v_head_dim=None) -> SagaDims:
+    """head_dim is the key (and query) head dim; v_head_dim the value head dim
+    (None: the same)."""
+    return SagaDims(batch, h_q, h_k, h_v, head_dim, l_kv, l_kv if l_cap is None else l_cap,
+                    0 if v_head_dim is None else v_head_dim)
 
 
 def status_string(status: int) -> str:

@@ -23,7 +23,7 @@ namespace saga {
 
 constexpr int kCombineThreads = 256;
 
-template <int D, int NT>
+template <int DV, int D, int NT>  // D: key/query head dim, DV: value head dim
 __device__ void fallback_row(const CombineArgs& a, long long row, float m_star, float* out_row,
                              int32_t* cnt_out, uint8_t* kbuf) {
     const Geometry& g = a.g;
@@ -34,8 +34,7 @@ __device__ void fallback_row(const CombineArgs& a, long long row, float m_star, 
     const int vh = i * g.hv / g.hq;
     const int nti = hl >> 3, col = hl & 7;
     const int gq = lane >> 2, tq = lane & 3;
-    constexpr int DH = D / 64;
-    constexpr int CPL = D / 32;  // value columns per lane
+    constexpr int CPL = DV / 32;  // value columns per lane
 
     QFrag<D, NT> qf;
     load_q_frag<D, NT>(qf, reinterpret_cast<const __nv_bfloat16*>(a.q), g.hq, g.G, bb, kh, lane);
@@ -49,13 +48,13 @@ __device__ void fallback_row(const CombineArgs& a, long long row, float m_star, 
         // 16 key rows of head kh into the swizzled tile layout of qk_mma
         for (int q8 = lane; q8 < 16 * D / 8; q8 += 32) {
             const int r = q8 / (D / 8), cc = q8 - r * (D / 8);
-            const int dh = cc >> 3, c8 = cc & 7;
+            const int dh = cc / KTile<D>::CPR, c8 = cc % KTile<D>::CPR;
             const int pos = j0 + r;
             uint4 v = make_uint4(0u, 0u, 0u, 0u);
             if (pos < g.l)
                 v = *reinterpret_cast<const uint4*>(
                     K + ((static_cast<size_t>(bb) * g.l_cap + pos) * g.hk + kh) * D + cc * 8);
-            *reinterpret_cast<uint4*>(kbuf + dh * 16 * 128 + r * 128 + ((c8 ^ (r & 7)) << 4)) = v;
+            *reinterpret_cast<uint4*>(kbuf + KTile<D>::offset(dh, 16, r, c8)) = v;
         }
         __syncwarp();
         float acc[1][NT][4];
@@ -78,7 +77,7 @@ __device__ void fallback_row(const CombineArgs& a, long long row, float m_star, 
                 ball &= ball - 1;
                 const int pos = j0 + (src >> 2) + 8 * h;
                 const __nv_bfloat16* vr =
-                    V + ((static_cast<size_t>(bb) * g.l_cap + pos) * g.hv + vh) * D + lane * CPL;
+                    V + ((static_cast<size_t>(bb) * g.l_cap + pos) * g.hv + vh) * DV + lane * CPL;
 #pragma unroll
                 for (int c = 0; c < CPL; ++c) osum[c] += __bfloat162float(vr[c]);
                 ++count;
@@ -88,7 +87,6 @@ __device__ void fallback_row(const CombineArgs& a, long long row, float m_star, 
 #pragma unroll
     for (int c = 0; c < CPL; ++c) out_row[lane * CPL + c] = osum[c] / static_cast<float>(count);
     if (lane == 0 && cnt_out) *cnt_out = count;
-    (void)DH;
 }
 
 // Number of partial records of row (of batch element bb).
@@ -104,7 +102,7 @@ __device__ __forceinline__ int row_records(const CombineArgs& a, int bb) {
 // (m, l, count, m_all, o) without normalising.  All kCombineThreads threads
 // of the block take part (block barriers).  Records are read through L2, so
 // a CTA of the kernel that wrote them may merge them.
-template <int D, int NT>
+template <int D, int DK, int NT>  // D: value head dim, DK: key/query head dim
 __device__ void combine_row(const CombineArgs& a, long long row, int r_begin = 0, int R = -1,
                             float* partial_out = nullptr) {
     constexpr int kWarps = kCombineThreads / 32;
@@ -112,7 +110,7 @@ __device__ void combine_row(const CombineArgs& a, long long row, int r_begin = 0
     __shared__ float red[3][kWarps];
     __shared__ int red_c[kWarps];
     __shared__ float red_o[kWarps][D];
-    __shared__ __align__(1024) uint8_t kbuf[16 * D * 2];
+    __shared__ __align__(1024) uint8_t kbuf[16 * DK * 2];
 
     const Geometry& g = a.g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -152,7 +150,7 @@ __device__ void combine_row(const CombineArgs& a, long long row, int r_begin = 0
     float* out_row = a.out + static_cast<size_t>(row) * D;
     if (cnt == 0 && a.fallback && !partial_out) {
         if (warp == 0)
-            fallback_row<D, NT>(a, row, mall, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf);
+            fallback_row<D, DK, NT>(a, row, mall, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf);
         return;
     }
 

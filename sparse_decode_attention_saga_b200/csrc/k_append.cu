@@ -19,15 +19,15 @@ namespace {
 __global__ void __launch_bounds__(256) append_kernel(const AppendArgs a) {
     pdl_wait();  // the cache may still be read by the previous step's kernels
     pdl_trigger();
-    const int chunks_row = a.d / 8;  // 16-byte chunks per head row
-    const long long nk = static_cast<long long>(a.b) * a.hk * chunks_row;
-    const long long nv = static_cast<long long>(a.b) * a.hv * chunks_row;
+    const int ck = a.d / 8, cv = a.dv / 8;  // 16-byte chunks per key / value head row
+    const long long nk = static_cast<long long>(a.b) * a.hk * ck;
+    const long long nv = static_cast<long long>(a.b) * a.hv * cv;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nk + nv;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         const bool is_k = i < nk;
         const long long j = is_k ? i : i - nk;
         const int heads = is_k ? a.hk : a.hv;
-        const long long per_b = static_cast<long long>(heads) * chunks_row;
+        const long long per_b = static_cast<long long>(heads) * (is_k ? ck : cv);
         const long long bb = j / per_b;
         const long long rem = j - bb * per_b;  // (head, chunk) inside the new row
         const uint4* src = reinterpret_cast<const uint4*>(is_k ? a.k_new : a.v_new) + j;
@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendArgs a) {
 }  // namespace
 
 cudaError_t launch_cache_append(const AppendArgs& a, cudaStream_t stream) {
-    const long long chunks = static_cast<long long>(a.b) * (a.hk + a.hv) * (a.d / 8);
+    const long long chunks = static_cast<long long>(a.b) * (a.hk * (a.d / 8) + a.hv * (a.dv / 8));
     const unsigned blocks = static_cast<unsigned>((chunks + 255) / 256 < 1024 ? (chunks + 255) / 256 : 1024);
     return launch_dependent(append_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, stream, a);
 }

@@ -28,23 +28,23 @@ namespace {
 // (the B-fragment reads of the eight heads then hit distinct banks)
 __host__ __device__ constexpr int weight_stride(int d) { return (128 / d) * 16 + 8; }
 
-template <int D, int NT, int NCT>
+template <int D, int DV, int NT, int NCT>  // D: key/query head dim, DV: value head dim
 __global__ void __launch_bounds__(kStreamThreads, 1)
     dense_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                  const DenseArgs a) {
     constexpr int MBW = 128 / D;
-    constexpr int DH = D / 64;
+    constexpr int DVH = DV / 64;       // 64-wide value boxes per value head
     constexpr int HS = NT * 8;         // head slots per key head
     constexpr int ROWS = MBW * 16;     // positions per warp per tile
     constexpr int PS = weight_stride(D);
-    constexpr int MT = D / 16;         // 16-dim row tiles of O^T
+    constexpr int MT = DV / 16;        // 16-dim row tiles of O^T
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     const Geometry& g = a.g;
     const int stages = a.stages;
-    const int vbytes = g.P * g.hv * D * 2;
+    const int vbytes = g.P * g.hv * DV * 2;
     const int stage_bytes = kStageBytes + vbytes;
     uint16_t* pbuf_all = reinterpret_cast<uint16_t*>(smem + static_cast<size_t>(stages) * stage_bytes);
     float* abuf_all = reinterpret_cast<float*>(pbuf_all + kConsumerWarps * 2 * HS * PS);
@@ -84,12 +84,12 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 mbar_arrive_expect_tx(&full[st], stage_bytes);
                 uint8_t* dst = smem + static_cast<size_t>(st) * stage_bytes;
                 for (int kh = 0; kh < g.hk; ++kh)
-                    for (int dh = 0; dh < DH; ++dh)
-                        tma_load_3d(dst + (kh * DH + dh) * g.P * 128, &kmap, &full[st], dh * 64,
-                                    kh, z);
+                    for (int dh = 0; dh < KTile<D>::NBOX; ++dh)
+                        tma_load_3d(dst + (kh * KTile<D>::NBOX + dh) * g.P * KTile<D>::ROWB, &kmap,
+                                    &full[st], dh * 64, kh, z);
                 for (int vh = 0; vh < g.hv; ++vh)
-                    for (int dh = 0; dh < DH; ++dh)
-                        tma_load_3d(dst + kStageBytes + (vh * DH + dh) * g.P * 128, &vmap,
+                    for (int dh = 0; dh < DVH; ++dh)
+                        tma_load_3d(dst + kStageBytes + (vh * DVH + dh) * g.P * 128, &vmap,
                                     &full[st], dh * 64, vh, z);
                 issued = k + 1;
             }
@@ -109,14 +109,14 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     uint16_t* pb_lo = pb_hi + HS * PS;
     float* abuf = abuf_all + warp * HS;
 
-    // Column tiles of O^T: NCT tiles of 8 head slots.  With two value heads
-    // per key head (VPK = 2) tile ct holds the GV <= 8 query heads of value
-    // head kh*2 + ct; otherwise the G heads of the group's one value head
-    // fill tiles of 8.
+    // Column tiles of O^T: NCT tiles of 8 head slots.  With VPK = 2 value
+    // heads per key head, tile ct holds the GV = G / 2 <= 8 query heads of
+    // value head kh*2 + ct; otherwise the G heads of the group's one value
+    // head fill tiles of 8.
     const int VPK = g.hv > g.hk ? g.hv / g.hk : 1;
     const int GV = G / VPK;
-    auto head_of = [&](int ct, int n) { return VPK == 2 ? ct * GV + n : ct * 8 + n; };
-    auto head_ok = [&](int ct, int n) { return VPK == 2 ? n < GV : ct * 8 + n < G; };
+    auto head_of = [&](int ct, int n) { return VPK > 1 ? ct * GV + n : ct * 8 + n; };
+    auto head_ok = [&](int ct, int n) { return VPK > 1 ? n < GV : ct * 8 + n < G; };
     int vh_ct[NCT];
 #pragma unroll
     for (int ct = 0; ct < NCT; ++ct) vh_ct[ct] = (kh * G + head_of(ct, 0)) * g.hv / g.hq;
@@ -294,9 +294,9 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 uint32_t a0 = 0u, a1 = 0u, a2 = 0u, a3 = 0u;
 #pragma unroll
                 for (int ct = 0; ct < NCT; ++ct) {
-                    if (ct == 0 || VPK == 2) {
+                    if (ct == 0 || VPK > 1) {
                         const uint32_t addr = sbase + kStageBytes +
-                                              static_cast<uint32_t>((vh_ct[ct] * DH + dh) * g.P * 128 + pos * 128 +
+                                              static_cast<uint32_t>((vh_ct[ct] * DVH + dh) * g.P * 128 + pos * 128 +
                                                                     ((chunk ^ (pos & 7)) << 4));
                         ldmatrix_x4_trans(addr, a0, a1, a2, a3);
                         if (ragged) {
@@ -322,11 +322,11 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
     if (!ok && lane == 0) raise_device_error(a.err, kErrTimeout);
 }
 
-template <int D, int NT, int NCT>
+template <int D, int DV, int NT, int NCT>
 cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, const DenseArgs& a,
                      cudaStream_t stream) {
     const size_t smem = dense_smem_bytes(a.g, a.stages);
-    auto kern = dense_kernel<D, NT, NCT>;
+    auto kern = dense_kernel<D, DV, NT, NCT>;
     static const cudaError_t attr = cudaFuncSetAttribute(
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem);
     if (attr != cudaSuccess) return attr;
@@ -339,11 +339,13 @@ cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, const Den
 
 bool dense_supported(const Geometry& g) {
     // each key head's query heads use one value head, or two whole ones
+    // (more value heads per key head would also not fit a stage: its value
+    // rows are the K tile's bytes times h_v*d_v / (h_k*d))
     return g.hv <= 2 * g.hk && (g.hv % g.hk == 0 || g.hk % g.hv == 0);
 }
 
 size_t dense_stage_bytes(const Geometry& g) {
-    return static_cast<size_t>(kStageBytes) + static_cast<size_t>(g.P) * g.hv * g.d * 2;
+    return static_cast<size_t>(kStageBytes) + static_cast<size_t>(g.P) * g.hv * g.dv * 2;
 }
 
 size_t dense_smem_bytes(const Geometry& g, int stages) {
@@ -356,14 +358,22 @@ size_t dense_smem_bytes(const Geometry& g, int stages) {
 cudaError_t launch_dense(const CUtensorMap& kmap, const CUtensorMap& vmap, const DenseArgs& a,
                          cudaStream_t stream) {
     if (!dense_supported(a.g)) return cudaErrorInvalidValue;
-    const int d = a.g.d, nt = a.g.NT;
-    const bool two = a.g.hv > a.g.hk || nt == 2;  // two column tiles of query heads
-    if (d == 64 && nt == 1) return two ? launch_t<64, 1, 2>(kmap, vmap, a, stream)
-                                       : launch_t<64, 1, 1>(kmap, vmap, a, stream);
-    if (d == 64 && nt == 2) return launch_t<64, 2, 2>(kmap, vmap, a, stream);
-    if (d == 128 && nt == 1) return two ? launch_t<128, 1, 2>(kmap, vmap, a, stream)
-                                        : launch_t<128, 1, 1>(kmap, vmap, a, stream);
-    if (d == 128 && nt == 2) return launch_t<128, 2, 2>(kmap, vmap, a, stream);
+    const int d = a.g.d, dv = a.g.dv, nt = a.g.NT;
+    const int vpk = a.g.hv > a.g.hk ? a.g.hv / a.g.hk : 1;
+    const int nct = vpk > 1 ? vpk : nt;  // column tiles of query heads: 1 or 2
+#define SAGA_DENSE_CASE(DK_, DV_, NT_, NCT_)                                   \
+    if (d == DK_ && dv == DV_ && nt == NT_ && nct == NCT_)                     \
+        return launch_t<DK_, DV_, NT_, NCT_>(kmap, vmap, a, stream);
+    SAGA_DENSE_CASE(64, 64, 1, 1)
+    SAGA_DENSE_CASE(64, 64, 1, 2)
+    SAGA_DENSE_CASE(64, 64, 2, 2)
+    SAGA_DENSE_CASE(128, 128, 1, 1)
+    SAGA_DENSE_CASE(128, 128, 1, 2)
+    SAGA_DENSE_CASE(128, 128, 2, 2)
+    SAGA_DENSE_CASE(32, 64, 1, 1)
+    SAGA_DENSE_CASE(32, 64, 1, 2)
+    SAGA_DENSE_CASE(32, 64, 2, 2)
+#undef SAGA_DENSE_CASE
     return cudaErrorInvalidValue;
 }
 

@@ -43,11 +43,10 @@ constexpr int kGatherMinBlocks = SAGA_GATHER_MINBLOCKS;
 
 static_assert(kThreads == kCombineThreads, "the last CTA of a row runs the row merge");
 
-template <int D, int NT>
+template <int D, int DK, int NT>  // D: value head dim, DK: key/query head dim
 __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(const GatherArgs a) {
     constexpr int LPR = D * 2 / 16;    // lanes per value row (16 B each)
     constexpr int RPI = 32 / LPR;      // value rows per warp instruction
-    constexpr int MBW = 128 / D;
 
     extern __shared__ int table[];     // pre, start, slot_pos, slot_len
     __shared__ float red_m[kWarps];
@@ -96,7 +95,7 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
             const long long s0 = t0 > x0 ? t0 : x0;
             const long long s1 = t1 < x0 + g.tiles ? t1 : x0 + g.tiles;
             slot_pos[sl] = static_cast<int>((s0 - x0) * g.P);
-            slot_len[sl] = static_cast<int>((s1 - s0) * MBW * 16);  // entries a warp can hold
+            slot_len[sl] = static_cast<int>((s1 - s0) * g.MBW * 16);  // entries a warp can hold
         }
         __syncthreads();
         // counts (coalesced reads), clamped to each list's capacity
@@ -280,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     if (!is_last) return;
     __threadfence();
     if (tid == 0) a.tickets[row] = 0u;
-    combine_row<D, NT>(a.cmb, row);
+    combine_row<D, DK, NT>(a.cmb, row);
 }
 
 }  // namespace
@@ -293,17 +292,20 @@ cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
     const dim3 grid(a.parts, static_cast<unsigned>(static_cast<long long>(a.g.b) * a.g.hq));
     const size_t smem = gather_smem_bytes(a.max_lists, a.max_slots);
     if (smem > static_cast<size_t>(kGatherMaxSmem) || a.cmb.parts != a.parts) return cudaErrorInvalidValue;
-#define SAGA_GATHER_CASE(D_, NT_)                                                                  \
-    if (a.g.d == D_ && a.g.NT == NT_) {                                                            \
-        static const cudaError_t attr = cudaFuncSetAttribute(                                     \
-            gather_pv_kernel<D_, NT_>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem); \
-        if (attr != cudaSuccess) return attr;                                                      \
-        return launch_dependent(gather_pv_kernel<D_, NT_>, grid, dim3(kThreads), smem, stream, a); \
+#define SAGA_GATHER_CASE(D_, DK_, NT_)                                                         \
+    if (a.g.dv == D_ && a.g.d == DK_ && a.g.NT == NT_) {                                       \
+        auto kern = gather_pv_kernel<D_, DK_, NT_>;                                            \
+        static const cudaError_t attr =                                                        \
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem); \
+        if (attr != cudaSuccess) return attr;                                                  \
+        return launch_dependent(kern, grid, dim3(kThreads), smem, stream, a);                  \
     }
-    SAGA_GATHER_CASE(64, 1)
-    SAGA_GATHER_CASE(64, 2)
-    SAGA_GATHER_CASE(128, 1)
-    SAGA_GATHER_CASE(128, 2)
+    SAGA_GATHER_CASE(64, 64, 1)
+    SAGA_GATHER_CASE(64, 64, 2)
+    SAGA_GATHER_CASE(128, 128, 1)
+    SAGA_GATHER_CASE(128, 128, 2)
+    SAGA_GATHER_CASE(64, 32, 1)
+    SAGA_GATHER_CASE(64, 32, 2)
 #undef SAGA_GATHER_CASE
     return cudaErrorInvalidValue;
 }

@@ -47,7 +47,6 @@ template <int D, int NT, int MODE>
 __global__ void __launch_bounds__(kStreamThreads, 2)
     qk_stream_kernel(const __grid_constant__ CUtensorMap kmap, const StreamArgs a) {
     constexpr int MBW = 128 / D;
-    constexpr int DH = D / 64;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -93,9 +92,9 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
                 mbar_arrive_expect_tx(&full[st], kStageBytes);
                 uint8_t* dst = smem + static_cast<size_t>(st) * kStageBytes;
                 for (int kh = 0; kh < g.hk; ++kh)
-                    for (int dh = 0; dh < DH; ++dh)
-                        tma_load_3d_hint(dst + (kh * DH + dh) * g.P * 128, &kmap, &full[st],
-                                         dh * 64, kh, z, k_policy);
+                    for (int dh = 0; dh < KTile<D>::NBOX; ++dh)
+                        tma_load_3d_hint(dst + (kh * KTile<D>::NBOX + dh) * g.P * KTile<D>::ROWB,
+                                         &kmap, &full[st], dh * 64, kh, z, k_policy);
                 issued = k + 1;
                 if (++tl == g.tiles) {
                     tl = 0;
@@ -342,6 +341,8 @@ cudaError_t launch_qk_stream(int mode, const CUtensorMap& kmap, const StreamArgs
     SAGA_QK_CASE(64, 2)
     SAGA_QK_CASE(128, 1)
     SAGA_QK_CASE(128, 2)
+    SAGA_QK_CASE(32, 1)
+    SAGA_QK_CASE(32, 2)
 #undef SAGA_QK_CASE
     return cudaErrorInvalidValue;
 }

@@ -11,15 +11,32 @@
 // C fragment of lane (g = lane/4, t = lane%4): c[0], c[1] = rows g, columns
 // 2t, 2t+1; c[2], c[3] = row g+8, same columns.
 //
-// Shared-memory K tile: one TMA box per (key head kh, 64-wide half dh of the
+// Shared-memory K tile: one TMA box per (key head kh, 64-wide part dh of the
 // head dim), [rows = positions][128 B], written with the 128-byte swizzle
-// (16-byte chunk c of row r lands at chunk c ^ (r & 7)), so the eight row
-// addresses of every ldmatrix phase hit distinct banks.
+// (16-byte chunk c of row r lands at chunk c ^ (r & 7)); 32-dim keys use
+// one box per head with 64-byte rows and the 64-byte swizzle (chunk c of
+// row r at c ^ ((r >> 1) & 3)).  Either way the eight row addresses of every
+// ldmatrix phase hit distinct banks.
 #pragma once
 
 #include "saga_device.cuh"
 
 namespace saga {
+
+// Shared-memory layout of the K boxes for head dim D.
+template <int D>
+struct KTile {
+    static constexpr int ROWB = D >= 64 ? 128 : D * 2;  // bytes per box row
+    static constexpr int NBOX = D >= 64 ? D / 64 : 1;   // boxes per key head
+    static constexpr int CPR = ROWB / 16;               // 16-byte chunks per row
+    static constexpr int BOXW = ROWB / 2;               // elements per box row
+    // byte offset of 16-byte chunk `chunk` (logical) of row r of box `box`
+    static __host__ __device__ __forceinline__ int offset(int box, int rows_per_box, int r,
+                                                          int chunk) {
+        const int swz = ROWB == 128 ? (r & 7) : ((r >> 1) & 3);
+        return box * rows_per_box * ROWB + r * ROWB + ((chunk ^ swz) << 4);
+    }
+};
 
 // q fragments of one key head's group: qf[nt][ks][0..1] for n-tile nt
 // (query heads nt*8 .. nt*8+7 of the group) and k-step ks (16 dims).
@@ -54,7 +71,7 @@ template <int D, int NT, int MB>
 __device__ __forceinline__ void qk_mma(uint32_t tile, int rows_per_box, int kh, int mb0,
                                        const QFrag<D, NT>& qf, float (&acc)[MB][NT][4],
                                        int lane) {
-    constexpr int DH = D / 64;
+    using L = KTile<D>;
     const int chunk_hi = lane >> 4;
 #pragma unroll
     for (int mbi = 0; mbi < MB; ++mbi) {
@@ -65,10 +82,10 @@ __device__ __forceinline__ void qk_mma(uint32_t tile, int rows_per_box, int kh, 
         const int r = (mb0 + mbi) * 16 + (lane & 15);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-            const int dh = ks >> 2;
-            const int chunk = ((ks & 3) << 1) | chunk_hi;
-            const uint32_t addr = tile + static_cast<uint32_t>((kh * DH + dh) * rows_per_box * 128 +
-                                                               r * 128 + ((chunk ^ (r & 7)) << 4));
+            const int dh = ks / (L::CPR / 2);  // 16 dims = two chunks per k-step
+            const int chunk = ((ks % (L::CPR / 2)) << 1) | chunk_hi;
+            const uint32_t addr =
+                tile + static_cast<uint32_t>(L::offset(kh * L::NBOX + dh, rows_per_box, r, chunk));
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4(addr, a0, a1, a2, a3);
 #pragma unroll

@@ -98,7 +98,13 @@ int make_geometry(const saga_dims* d, Geometry* g) {
     if (d->batch <= 0 || d->h_q <= 0 || d->h_k <= 0 || d->h_v <= 0 || d->head_dim <= 0 ||
         d->l_kv <= 0 || d->l_cap < d->l_kv)
         return SAGA_ERR_INVALID_ARG;
-    if (d->head_dim != 64 && d->head_dim != 128) return SAGA_ERR_UNSUPPORTED;
+    if (d->v_head_dim < 0) return SAGA_ERR_INVALID_ARG;
+    const int dv = d->v_head_dim ? d->v_head_dim : d->head_dim;
+    // key/value head dims: equal and 64 or 128, or 32-dim keys with 64-dim
+    // values (two or more key heads, so that a 32 KB tile has <= 256 rows)
+    const bool same = (d->head_dim == 64 || d->head_dim == 128) && dv == d->head_dim;
+    const bool narrow_keys = d->head_dim == 32 && dv == 64 && d->h_k >= 2;
+    if (!same && !narrow_keys) return SAGA_ERR_UNSUPPORTED;
     if (d->h_k != 1 && d->h_k != 2 && d->h_k != 4 && d->h_k != 8) return SAGA_ERR_UNSUPPORTED;
     if (d->h_q % d->h_k != 0 || d->h_q % d->h_v != 0) return SAGA_ERR_UNSUPPORTED;
     if (d->h_q / d->h_k > 16 || d->h_q > 128) return SAGA_ERR_UNSUPPORTED;
@@ -110,11 +116,13 @@ int make_geometry(const saga_dims* d, Geometry* g) {
     x.hk = d->h_k;
     x.hv = d->h_v;
     x.d = d->head_dim;
+    x.dv = dv;
     x.l = d->l_kv;
     x.l_cap = d->l_cap;
     x.G = x.hq / x.hk;
     x.NT = (x.G + 7) / 8;
     x.P = kStageBytes / (x.hk * x.d * 2);
+    x.KB = x.d < 64 ? x.d : 64;
     x.WPK = kConsumerWarps / x.hk;
     x.MBW = 128 / x.d;
     x.tiles = (x.l + x.P - 1) / x.P;
@@ -123,7 +131,7 @@ int make_geometry(const saga_dims* d, Geometry* g) {
     // C <= b*tiles (every range holds at least floor(T/C) >= T/(2C) tiles).
     const int per_batch = 2 * ((kMaxCtas + x.b - 1) / x.b) + 2;
     x.S_cap = per_batch < x.tiles ? per_batch : x.tiles;
-    x.rec = x.d + kRecHeader;
+    x.rec = x.dv + kRecHeader;
     x.scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(x.d)));
     return SAGA_OK;
 }
@@ -139,17 +147,20 @@ T* ws_at(void* ws, size_t off) {
     return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-int encode_cache_map(CUtensorMap* map, const void* base, const Geometry& g, int heads,
-                     bool swizzle) {
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(heads),
+// Tensor map of a cache [b * l_cap, heads, dim] bf16: boxes of min(dim, 64)
+// elements x 1 head x P positions, each box row swizzled across its width
+// (128-byte rows for 64-element boxes, 64-byte rows for 32-dim keys).
+int encode_cache_map(CUtensorMap* map, const void* base, const Geometry& g, int heads, int dim) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(dim), static_cast<cuuint64_t>(heads),
                           static_cast<cuuint64_t>(g.b) * g.l_cap};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(g.d) * 2,
-                             static_cast<cuuint64_t>(heads) * g.d * 2};
-    cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(g.P)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(dim) * 2,
+                             static_cast<cuuint64_t>(heads) * dim * 2};
+    const cuuint32_t inner = dim < 64 ? static_cast<cuuint32_t>(dim) : 64u;
+    cuuint32_t box[3] = {inner, 1, static_cast<cuuint32_t>(g.P)};
     cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
                                 dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                inner == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? SAGA_OK : SAGA_ERR_CUDA;
@@ -231,7 +242,7 @@ void ev_stop(cudaStream_t s) {
 int run_logits(const Geometry& g, const DeviceInfo& dev, const void* q, const void* k, float* dst,
                uint32_t* err, cudaStream_t s) {
     CUtensorMap kmap;
-    int st = encode_cache_map(&kmap, k, g, g.hk, true);
+    int st = encode_cache_map(&kmap, k, g, g.hk, g.d);
     if (st) return st;
     StreamArgs a{};
     a.g = g;
@@ -384,7 +395,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     if (gather_smem_bytes(slots * g.WPK, slots) > static_cast<size_t>(kGatherMaxSmem))
         return SAGA_ERR_UNSUPPORTED;  // checked before anything is enqueued
     CUtensorMap kmap;
-    if ((st = encode_cache_map(&kmap, k, g, g.hk, true))) return st;
+    if ((st = encode_cache_map(&kmap, k, g, g.hk, g.d))) return st;
     StreamArgs a{};
     a.g = g;
     a.C = C;
@@ -448,8 +459,8 @@ int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const
     if (dense_smem_bytes(g, stages) > static_cast<size_t>(dev.max_smem)) return SAGA_ERR_UNSUPPORTED;
 
     CUtensorMap kmap, vmap;
-    if ((st = encode_cache_map(&kmap, k, g, g.hk, true))) return st;
-    if ((st = encode_cache_map(&vmap, v, g, g.hv, true))) return st;
+    if ((st = encode_cache_map(&kmap, k, g, g.hk, g.d))) return st;
+    if ((st = encode_cache_map(&vmap, v, g, g.hv, g.dv))) return st;
     DenseArgs a{};
     a.g = g;
     a.C = stream_ctas(g, dev, 1);
@@ -499,6 +510,7 @@ int saga_cache_append(const saga_dims* dims, const void* k_new, const void* v_ne
     a.hk = g.hk;
     a.hv = g.hv;
     a.d = g.d;
+    a.dv = g.dv;
     a.l_cap = g.l_cap;
     a.pos = g.l;
     a.k_new = k_new;

@@ -165,7 +165,7 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
 // Cache growth: new rows k_new [b,h_k,d], v_new [b,h_v,d] -> row `pos` of
 // k [b,l_cap,h_k,d] and v [b,l_cap,h_v,d].
 struct AppendArgs {
-    int b, hk, hv, d, l_cap, pos;
+    int b, hk, hv, d, dv, l_cap, pos;  // d: key head dim, dv: value head dim
     const void* k_new;
     const void* v_new;
     void* k;

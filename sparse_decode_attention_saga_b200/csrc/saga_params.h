@@ -39,15 +39,17 @@ constexpr int kRecHeader = 4;
 
 struct Geometry {
     int b, hq, hk, hv, d, l, l_cap;
+    int dv;     // value head dim (d is the key and query head dim)
     int G;      // query heads per key head
     int NT;     // n-tiles of 8 query heads per key head (1 or 2)
     int P;      // positions per tile: kStageBytes / (h_k * d * 2)
+    int KB;     // key TMA box / shared-memory row: min(d, 64) elements
     int WPK;    // consumer warps per key head: 8 / h_k
-    int MBW;    // 16-position m-blocks per warp per tile: 128 / d
+    int MBW;    // 16-position m-blocks per warp per tile: 128 / d (4 for d = 32)
     int tiles;  // tiles per batch row: ceil(l / P)
     int l_pad;  // tiles * P (row stride of the kept-entry lists)
     int S_cap;  // partial-record slots per (batch, query head)
-    int rec;    // floats per partial record: d + kRecHeader
+    int rec;    // floats per partial record: dv + kRecHeader
     float scale;
 };
 

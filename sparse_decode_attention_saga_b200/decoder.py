@@ -19,20 +19,22 @@ class AtopNDecoder:
     l_cap; ``append`` adds the step's own key/value rows (the cached length
     grows by one), so buffers are sized for l_cap."""
 
-    def __init__(self, batch, h_q, h_k, h_v, head_dim, l_kv, N, n, l_cap=None, device="cuda"):
+    def __init__(self, batch, h_q, h_k, h_v, head_dim, l_kv, N, n, l_cap=None, device="cuda",
+                 v_head_dim=None):
         self.l_cap = int(l_kv if l_cap is None else l_cap)
-        self.dims = _lib.dims(batch, h_q, h_k, h_v, head_dim, l_kv, self.l_cap)
+        self.dv = int(head_dim if v_head_dim is None else v_head_dim)
+        self.dims = _lib.dims(batch, h_q, h_k, h_v, head_dim, l_kv, self.l_cap, self.dv)
         self.N, self.n = int(N), int(n)
         self.device = torch.device(device)
         # a workspace sized for the full capacity serves every shorter length
         nbytes = _lib.workspace_bytes(_lib.dims(batch, h_q, h_k, h_v, head_dim, self.l_cap,
-                                                self.l_cap), self.N)
+                                                self.l_cap, self.dv), self.N)
         if nbytes == 0:
             raise _lib.SagaError("saga_workspace_bytes", _lib.SAGA_ERR_UNSUPPORTED)
         self.ws = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
         self.thresh = torch.full((batch, h_q), float("nan"), dtype=torch.float32, device=self.device)
         self._logits = torch.empty(batch * h_q * self.l_cap, dtype=torch.float32, device=self.device)
-        self.out = torch.empty((batch, h_q, head_dim), dtype=torch.float32, device=self.device)
+        self.out = torch.empty((batch, h_q, self.dv), dtype=torch.float32, device=self.device)
 
     @property
     def l_kv(self) -> int:
@@ -45,15 +47,17 @@ class AtopNDecoder:
         return self._logits[: d.batch * d.h_q * d.l_kv].view(d.batch, d.h_q, d.l_kv)
 
     def append(self, k_new, v_new, k, v, stream=None) -> None:
-        """Writes this step's key/value rows ([b,h_k,d], [b,h_v,d] bf16) at
+        """Writes this step's key/value rows ([b,h_k,d], [b,h_v,d_v] bf16) at
         position l_kv of the caches; the following steps see l_kv + 1 rows."""
         _lib.cache_append(self.dims, k_new, v_new, k, v, stream)
         d = self.dims
-        self.dims = _lib.dims(d.batch, d.h_q, d.h_k, d.h_v, d.head_dim, d.l_kv + 1, self.l_cap)
+        self.dims = _lib.dims(d.batch, d.h_q, d.h_k, d.h_v, d.head_dim, d.l_kv + 1, self.l_cap,
+                              self.dv)
 
     @classmethod
     def for_workload(cls, w, device="cuda"):
-        return cls(w.batch, w.h_q, w.h_k, w.h_v, w.head_dim, w.l_kv, w.N, w.n, w.cap, device)
+        return cls(w.batch, w.h_q, w.h_k, w.h_v, w.head_dim, w.l_kv, w.N, w.n, w.cap, device,
+                   w.dv)
 
     def is_refresh(self, t: int) -> bool:
         return t % self.n == 0

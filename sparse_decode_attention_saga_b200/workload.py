@@ -38,10 +38,15 @@ class Workload:
     n: int
     steps: int = 32
     l_cap: int | None = None
+    v_head_dim: int | None = None  # value head dim where it differs from head_dim
 
     @property
     def cap(self) -> int:
         return self.l_kv if self.l_cap is None else self.l_cap
+
+    @property
+    def dv(self) -> int:
+        return self.head_dim if self.v_head_dim is None else self.v_head_dim
 
     def scaled(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -94,16 +99,16 @@ def topic_vectors(w: Workload, seed: int, device="cpu") -> torch.Tensor:
 
 
 def make_cache(w: Workload, seed: int = 0, device="cpu"):
-    """Returns (K [b,l_cap,h_k,d] bf16, V [b,l_cap,h_v,d] bf16).
+    """Returns (K [b,l_cap,h_k,d] bf16, V [b,l_cap,h_v,d_v] bf16).
 
     Drawn one batch element at a time so the fp32 temporaries stay small.
     Rows at positions >= l_kv (spare capacity) are drawn like the others.
     """
     u = topic_vectors(w, seed, device)
     g = _gen(seed * 7919 + 2, device)
-    b, L, hk, hv, d = w.batch, w.cap, w.h_k, w.h_v, w.head_dim
+    b, L, hk, hv, d, dv = w.batch, w.cap, w.h_k, w.h_v, w.head_dim, w.dv
     K = torch.empty(b, L, hk, d, dtype=torch.bfloat16, device=device)
-    V = torch.empty(b, L, hv, d, dtype=torch.bfloat16, device=device)
+    V = torch.empty(b, L, hv, dv, dtype=torch.bfloat16, device=device)
     n_topic = max(1, int(round(TOPIC_FRACTION * w.l_kv)))
     for bb in range(b):
         kf = torch.randn(L, hk, d, generator=g, device=device, dtype=torch.float32)
@@ -112,7 +117,7 @@ def make_cache(w: Workload, seed: int = 0, device="cpu"):
             kf[pos, kh, :] += TOPIC_SHIFT * u[kh]
         K[bb] = kf.to(torch.bfloat16)
         del kf
-        V[bb] = torch.randn(L, hv, d, generator=g, device=device,
+        V[bb] = torch.randn(L, hv, dv, generator=g, device=device,
                             dtype=torch.float32).to(torch.bfloat16)
     return K, V
 
@@ -131,7 +136,7 @@ def make_queries(w: Workload, seed: int = 0, device="cpu", steps: int | None = N
 
 def make_new_rows(w: Workload, seed: int = 0, device="cpu", steps: int | None = None):
     """Key and value rows generated one per decode step, for a growing cache:
-    ([steps, b, h_k, d], [steps, b, h_v, d]) bf16, drawn like the cache rows
+    ([steps, b, h_k, d], [steps, b, h_v, d_v]) bf16, drawn like the cache rows
     (N(0,1); each (step, batch, key head) key row gets 2*u_k added with
     probability 2 %)."""
     steps = w.steps if steps is None else steps
@@ -141,7 +146,7 @@ def make_new_rows(w: Workload, seed: int = 0, device="cpu", steps: int | None = 
                      dtype=torch.float32)
     shift = torch.rand(steps, w.batch, w.h_k, generator=g, device=device) < TOPIC_FRACTION
     kf += TOPIC_SHIFT * shift[..., None].float() * u[None, None]
-    vf = torch.randn(steps, w.batch, w.h_v, w.head_dim, generator=g, device=device,
+    vf = torch.randn(steps, w.batch, w.h_v, w.dv, generator=g, device=device,
                      dtype=torch.float32)
     return kf.to(torch.bfloat16), vf.to(torch.bfloat16)
 

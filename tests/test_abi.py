@@ -141,3 +141,16 @@ def test_cache_append_validation(lib):
     bad = _lib.dims(1, 4, 1, 2, 96, 64, 65)
     assert lib.saga_cache_append(ctypes.byref(bad), 16, 16, 16, 16, None) == \
         _lib.SAGA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("hk,d,dv,ok", [
+    (2, 32, 64, True),     # Sigma-style keys: 32 dims, values 64
+    (1, 32, 64, False),    # one key head: a 32 KB tile would need 512 rows
+    (2, 32, 128, False),
+    (2, 64, 32, False),
+    (2, 64, 128, False),
+    (2, 128, 0, True),     # 0: values share the key dim
+])
+def test_value_head_dim_validation(lib, hk, d, dv, ok):
+    dims = _lib.dims(1, 16, hk, 8, d, 256, None, dv)
+    assert (_lib.workspace_bytes(dims, 8) > 0) == ok

@@ -125,6 +125,31 @@ def test_N_at_least_l_is_full_attention(hq, hk, hv, d):
     np.testing.assert_allclose(dense, ref_attention(qs[0], K, V, w.l_kv), rtol=1e-5, atol=1e-6)
 
 
+def test_narrow_keys_sigma_layout_is_attention_with_separate_head_dims():
+    """Keys (and queries) of 32 dims, values of 64 (the pages' Sigma-style
+    (h_k, d_k) = (2, 32) next to h_v = 8, d_v = 64): the logits scale by
+    1/sqrt(32) and the output has the value dim.  Full attention (N >= l)
+    against library float64 attention, and a reuse step against library
+    attention restricted to the oracle's mask."""
+    w = Workload("sigma", 2, 16, 2, 8, 32, 180, 180, 4, steps=2, v_head_dim=64)
+    qs, K, V = inputs(w, seed=13)
+    assert qs.shape[-1] == 32 and K.shape[-1] == 32 and V.shape[-1] == 64
+    tau = np.zeros((w.batch, w.h_q), np.float32)
+    out, s, mask, cnt = oracle.atopn_step(bf16_bits(qs[0]), bf16_bits(K), bf16_bits(V), tau,
+                                          w.l_kv, 0, 4)
+    assert out.shape == (w.batch, w.h_q, 64)
+    np.testing.assert_allclose(out, ref_attention(qs[0], K, V, w.l_kv), rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(s, ref_logits64(qs[0], K, w.l_kv), rtol=1e-6, atol=1e-6)
+    dense = oracle.decode_dense(bf16_bits(qs[0]), bf16_bits(K), bf16_bits(V))
+    np.testing.assert_allclose(dense, ref_attention(qs[0], K, V, w.l_kv), rtol=1e-5, atol=1e-6)
+    tau = np.zeros((w.batch, w.h_q), np.float32)
+    oracle.atopn_step(bf16_bits(qs[0]), bf16_bits(K), bf16_bits(V), tau, 12, 0, 4)  # refresh
+    out1, s1, mask1, _ = oracle.atopn_step(bf16_bits(qs[1]), bf16_bits(K), bf16_bits(V), tau,
+                                           12, 1, 4)                                 # reuse
+    np.testing.assert_allclose(out1, ref_attention(qs[1], K, V, w.l_kv, mask=mask1),
+                               rtol=1e-5, atol=1e-6)
+
+
 def test_hk_equal_hv_is_grouped_query_attention():
     w = small(hq=8, hk=2, hv=2, d=64, l=120)
     qs, K, V = inputs(w, seed=6)
