@@ -79,6 +79,10 @@ CONFIGS: dict[str, Workload] = {
     "llama_b16_128k": Workload("llama_b16_128k", 16, 32, 4, 8, 64, 131072, 2048, 16),
     **_headcount(),
     **_sweep(),
+    # keys narrower than values (the pages' Sigma-style head layout: (h_k, d_k)
+    # = (2, 32) next to h_v = 8, d_v = 64, h_q 16), batch 16, 128K context
+    "sigma_b16_128k": Workload("sigma_b16_128k", 16, 16, 2, 8, 32, 131072, 2048, 16,
+                               v_head_dim=64),
 }
 
 TOPIC_FRACTION = 0.02

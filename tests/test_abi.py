@@ -115,7 +115,7 @@ def test_valid_call_without_a_device_reports_no_device(lib):
 
 def test_workspace_sizes_for_every_workload(lib):
     for name, w in CONFIGS.items():
-        d = _lib.dims(w.batch, w.h_q, w.h_k, w.h_v, w.head_dim, w.l_kv, w.cap)
+        d = _lib.dims(w.batch, w.h_q, w.h_k, w.h_v, w.head_dim, w.l_kv, w.cap, w.dv)
         n = _lib.workspace_bytes(d, w.N)
         assert 0 < n < 4 << 30, name
 
