@@ -219,4 +219,81 @@ __device__ void combine_row(const CombineArgs& a, long long row, int r_begin = 0
     }
 }
 
+// Merge of R partial records that were all weighted with the same
+// reference (the row's largest logit m_all; empty records hold l = 0 and
+// o = 0): out = sum_r o_r / sum_r l_r, with every record load in flight at
+// once (one L2 round trip instead of the three dependent passes of
+// combine_row).  Rows that kept nothing take the empty-set fallback.
+template <int D, int DK, int NT>
+__device__ void merge_same_reference(const CombineArgs& a, long long row, int R, float m_all) {
+    constexpr int kWarps = kCombineThreads / 32;
+    constexpr int U = 4;  // records per warp
+    constexpr int CPL = D / 32;
+    __shared__ float red_o[kWarps][D];
+    __shared__ float red_l[kWarps];
+    __shared__ int red_c[kWarps];
+    __shared__ __align__(1024) uint8_t kbuf[16 * DK * 2];
+
+    const Geometry& g = a.g;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float* recs = a.records + static_cast<size_t>(row) * g.S_cap * g.WPK * g.rec;
+    float lw = 0.f, osum[CPL];
+    int cw = 0;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) osum[k] = 0.f;
+    for (int r0 = warp; r0 < R; r0 += U * kWarps) {  // one pass when R <= 32
+        float o[U][CPL], l[U];
+        int c[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int r = r0 + u * kWarps;
+            const float* rec = recs + static_cast<size_t>(r < R ? r : 0) * g.rec;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) o[u][k] = r < R ? __ldcg(rec + kRecHeader + lane * CPL + k) : 0.f;
+            l[u] = r < R ? __ldcg(rec + 1) : 0.f;
+            c[u] = r < R ? __float_as_int(__ldcg(rec + 2)) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            lw += l[u];
+            cw += c[u];
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) osum[k] += o[u][k];
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) red_o[warp][lane * CPL + k] = osum[k];
+    if (lane == 0) {
+        red_l[warp] = lw;
+        red_c[warp] = cw;
+    }
+    __syncthreads();
+    float lsum = 0.f;
+    int cnt = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        lsum += red_l[w];
+        cnt += red_c[w];
+    }
+    float* out_row = a.out + static_cast<size_t>(row) * D;
+    if (cnt == 0) {
+        if (a.fallback) {
+            if (warp == 0)
+                fallback_row<D, DK, NT>(a, row, m_all, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf);
+        } else {
+            for (int k = tid; k < D; k += kCombineThreads) out_row[k] = 0.f;
+            if (tid == 0 && a.sel_cnt) a.sel_cnt[row] = 0;
+        }
+        return;
+    }
+    const float inv = 1.f / lsum;
+    for (int k = tid; k < D; k += kCombineThreads) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) v += red_o[w][k];
+        out_row[k] = v * inv;
+    }
+    if (tid == 0 && a.sel_cnt) a.sel_cnt[row] = cnt;
+}
+
 }  // namespace saga

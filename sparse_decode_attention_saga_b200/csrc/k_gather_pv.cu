@@ -10,9 +10,13 @@
 // logit) pairs: one contiguous list from the compare/compact kernel
 // (kListContiguous), or one list per
 // (streaming CTA slot, consumer warp) from the fused kernel (kListSegments).
-// Grid (parts, rows): every CTA builds the row's list table (counts and
-// exclusive prefix) in shared memory and takes an equal share of the row's
-// flattened entries, so the work is balanced whatever the lists' lengths.
+// Grid (parts, rows), or (rows, parts) with part_major: every CTA builds the
+// row's list table (counts and exclusive prefix) in shared memory and takes
+// an equal share of the row's flattened entries, so the work is balanced
+// whatever the lists' lengths.  Parts past what the row's entry count needs
+// return without a record; with few rows (many parts per row) the grid is
+// part-major, so part p of every row is scheduled before part p + 1 of any
+// row and no row waits for a second wave of CTAs that turn out to be empty.
 // Each warp then works through its own contiguous part of that share without
 // block barriers: 32 entries at a time, one (position, logit) per lane read
 // with coalesced loads one round ahead, and 16-byte value-row loads by lane
@@ -20,7 +24,8 @@
 // fp32.  m is the row's largest logit, which is always kept when anything is
 // (tau_eff <= max), so no running max is needed.  The share's (m, sum of
 // weights, count, row max, unnormalised output) record is merged across
-// shares by the combine kernel.
+// shares by the last CTA of the row; all shares used the same reference m,
+// so the merge is a plain sum of the records in one pass.
 #include "combine_row.cuh"
 
 namespace saga {
@@ -43,7 +48,8 @@ constexpr int kGatherMinBlocks = SAGA_GATHER_MINBLOCKS;
 
 static_assert(kThreads == kCombineThreads, "the last CTA of a row runs the row merge");
 
-template <int D, int DK, int NT>  // D: value head dim, DK: key/query head dim
+// D: value head dim, DK: key/query head dim, PM: part-major grid (rows, parts)
+template <int D, int DK, int NT, bool PM>
 __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(const GatherArgs a) {
     constexpr int LPR = D * 2 / 16;    // lanes per value row (16 B each)
     constexpr int RPI = 32 / LPR;      // value rows per warp instruction
@@ -60,8 +66,8 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     pdl_trigger();
     const Geometry& g = a.g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const long long row = blockIdx.y;
-    const int part = blockIdx.x;
+    const long long row = PM ? blockIdx.x : blockIdx.y;
+    const int part = PM ? blockIdx.y : blockIdx.x;
     const int bb = static_cast<int>(row / g.hq);
     const int i = static_cast<int>(row - static_cast<long long>(bb) * g.hq);
     const int vh = i * g.hv / g.hq;
@@ -88,6 +94,11 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
         const int c_first = cta_of_tile(x0, T, a.C);
         const int slots = cta_of_tile(x0 + g.tiles - 1, T, a.C) - c_first + 1;
         nl = slots * g.WPK;  // <= max_lists (checked by the host)
+        // the first list's count and maximum are requested before the slot
+        // table is built, so their latency overlaps it
+        const size_t rbase = static_cast<size_t>(row) * g.S_cap * g.WPK;
+        const int cu_first = tid < nl ? a.seg_cnt[rbase + tid] : 0;
+        const float mall_first = tid < nl ? a.seg_mall[rbase + tid] : -kInf;
         // per-slot position offset and tile count of the streaming CTA's segment
         for (int sl = tid; sl < slots; sl += kThreads) {
             const int c = c_first + sl;
@@ -99,15 +110,14 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
         }
         __syncthreads();
         // counts (coalesced reads), clamped to each list's capacity
-        const size_t rbase = static_cast<size_t>(row) * g.S_cap * g.WPK;
         float mloc = -kInf;
         for (int j = tid; j < nl; j += kThreads) {
-            const int cu = a.seg_cnt[rbase + j];
+            const int cu = j == tid ? cu_first : a.seg_cnt[rbase + j];
             const int sl = j / g.WPK;
             const int cap = slot_len[sl];
             start[j] = slot_pos[sl] + (j - sl * g.WPK) * cap;
             pre[j] = cu < 0 ? 0 : (cu > cap ? cap : cu);
-            mloc = fmaxf(mloc, a.seg_mall[rbase + j]);
+            mloc = fmaxf(mloc, j == tid ? mall_first : a.seg_mall[rbase + j]);
         }
         __syncthreads();
         // exclusive scan: each thread owns a run of consecutive lists
@@ -145,12 +155,13 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
         __syncthreads();
     }
     const int total = pre[nl];
-    // Shares of at least kMinShare entries: with few kept entries per row most
-    // of the launched parts stay empty (their records say so) instead of each
-    // paying a CTA's fixed cost for a handful of rows.
+    // Shares of at least kMinShare entries: with few kept entries per row the
+    // parts past `parts` return here instead of each paying a CTA's fixed cost
+    // for a handful of rows.
     const int parts = max(1, min(a.parts, (total + kMinShare - 1) / kMinShare));
-    const int e0 = part < parts ? static_cast<int>(static_cast<long long>(total) * part / parts) : total;
-    const int e1 = part < parts ? static_cast<int>(static_cast<long long>(total) * (part + 1) / parts) : total;
+    if (part >= parts) return;  // not needed for this row: no record, no ticket
+    const int e0 = static_cast<int>(static_cast<long long>(total) * part / parts);
+    const int e1 = static_cast<int>(static_cast<long long>(total) * (part + 1) / parts);
     const int n = e1 - e0;
     // each warp owns a contiguous sub-share and needs no block barrier
     const int w0 = e0 + static_cast<int>(static_cast<long long>(n) * warp / kWarps);
@@ -271,15 +282,15 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
         rec[3] = m_all;
     }
 
-    // the row's last CTA to finish merges the row's records
+    // the row's last CTA to finish merges the row's `parts` records
     __threadfence();
     __syncthreads();
-    if (tid == 0) is_last = atomicAdd(a.tickets + row, 1u) == gridDim.x - 1;
+    if (tid == 0) is_last = atomicAdd(a.tickets + row, 1u) == static_cast<unsigned>(parts - 1);
     __syncthreads();
     if (!is_last) return;
     __threadfence();
     if (tid == 0) a.tickets[row] = 0u;
-    combine_row<D, DK, NT>(a.cmb, row);
+    merge_same_reference<D, DK, NT>(a.cmb, row, parts, m_all);
 }
 
 }  // namespace
@@ -288,17 +299,33 @@ size_t gather_smem_bytes(int max_lists, int max_slots) {
     return (2 * static_cast<size_t>(max_lists) + 1 + 2 * static_cast<size_t>(max_slots)) * sizeof(int);
 }
 
+// Lets both block orders of one instantiation use the list table's
+// dynamic shared memory (set once per instantiation).
+template <typename K>
+cudaError_t allow_table_smem(K k_rows, K k_parts) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem);
+    return e != cudaSuccess
+               ? e
+               : cudaFuncSetAttribute(k_parts, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem);
+}
+
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
-    const dim3 grid(a.parts, static_cast<unsigned>(static_cast<long long>(a.g.b) * a.g.hq));
+    const long long rows = static_cast<long long>(a.g.b) * a.g.hq;
+    if (a.parts < 1 || a.parts > 65535 || rows > (a.part_major ? 0x7fffffffll : 65535ll))
+        return cudaErrorInvalidValue;
+    const dim3 grid = a.part_major ? dim3(static_cast<unsigned>(rows), static_cast<unsigned>(a.parts))
+                                   : dim3(static_cast<unsigned>(a.parts), static_cast<unsigned>(rows));
     const size_t smem = gather_smem_bytes(a.max_lists, a.max_slots);
     if (smem > static_cast<size_t>(kGatherMaxSmem) || a.cmb.parts != a.parts) return cudaErrorInvalidValue;
 #define SAGA_GATHER_CASE(D_, DK_, NT_)                                                         \
     if (a.g.dv == D_ && a.g.d == DK_ && a.g.NT == NT_) {                                       \
-        auto kern = gather_pv_kernel<D_, DK_, NT_>;                                            \
-        static const cudaError_t attr =                                                        \
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem); \
+        auto k_rows = gather_pv_kernel<D_, DK_, NT_, false>;                                   \
+        auto k_parts = gather_pv_kernel<D_, DK_, NT_, true>;                                   \
+        static const cudaError_t attr = allow_table_smem(k_rows, k_parts);                     \
         if (attr != cudaSuccess) return attr;                                                  \
-        return launch_dependent(kern, grid, dim3(kThreads), smem, stream, a);                  \
+        return launch_dependent(a.part_major ? k_parts : k_rows, grid, dim3(kThreads), smem,   \
+                                stream, a);                                                    \
     }
     SAGA_GATHER_CASE(64, 64, 1)
     SAGA_GATHER_CASE(64, 64, 2)

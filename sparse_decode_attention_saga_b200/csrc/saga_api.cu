@@ -193,6 +193,12 @@ int stream_ctas(const Geometry& g, const DeviceInfo& dev, int per_sm) {
 
 // CTAs per row of the gather kernel: about 8 per SM over all rows, never more
 // than the partial-record slots of a row.
+// From this many CTAs per row (few rows) the gather grid is part-major: most
+// rows then need only some of their parts, and the needed ones go first
+// (measured: Llama-shaped batch 1 at 8K, 23.5 -> 21.5 us per reuse step;
+// row-major stays faster at batch 16, 233 -> 229 us).
+constexpr int kPartMajorParts = 16;
+
 int gather_parts(const Geometry& g, const DeviceInfo& dev) {
     const long long rows = static_cast<long long>(g.b) * g.hq;
     long long parts = (8ll * dev.sms + rows - 1) / rows;
@@ -370,6 +376,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         ga.g = g;
         ga.mode = kListContiguous;
         ga.parts = gather_parts(g, dev);
+        ga.part_major = ga.parts >= kPartMajorParts;
         ga.max_lists = 1;
         ga.max_slots = 1;
         ga.v = v;
@@ -417,6 +424,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     ga.mode = kListSegments;
     ga.C = a.C;
     ga.parts = gather_parts(g, dev);
+    ga.part_major = ga.parts >= kPartMajorParts;
     ga.max_slots = slots;
     ga.max_lists = slots * g.WPK;
     ga.v = v;

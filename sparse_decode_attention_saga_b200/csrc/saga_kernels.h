@@ -123,6 +123,7 @@ struct GatherArgs {
     Geometry g;
     int mode;
     int parts;      // CTAs per row (each takes an equal share of the row's entries)
+    int part_major; // grid (rows, parts) instead of (parts, rows)
     int C;          // kListSegments: grid of the fused kernel
     int max_lists;  // lists per row at most (kListSegments: slots * WPK; else 1)
     int max_slots;  // kListSegments: streaming-CTA slots per row at most; else 1
