@@ -63,7 +63,10 @@ def run_profile_case(args):
     dec = AtopNDecoder.for_workload(w)
     for t in range(3):
         dec.step(t, qs[t], K, V)
-    dec.dense(qs[0], K, V)
+    try:
+        dec.dense(qs[0], K, V)
+    except _lib.SagaError:  # shapes the dense kernel does not take
+        pass
     torch.cuda.synchronize()
     assert dec.error() == _lib.SAGA_OK
     return 0

@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     constexpr int LPR = D * 2 / 16;    // lanes per value row (16 B each)
     constexpr int RPI = 32 / LPR;      // value rows per warp instruction
 
-    extern __shared__ int table[];     // pre, start, slot_pos, slot_len
+    extern __shared__ int table[];     // pre, start
     __shared__ float red_m[kWarps];
     __shared__ float red_l[kWarps];
     __shared__ float red_o[kWarps][D];
@@ -71,10 +71,8 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     const int bb = static_cast<int>(row / g.hq);
     const int i = static_cast<int>(row - static_cast<long long>(bb) * g.hq);
     const int vh = i * g.hv / g.hq;
-    int* pre = table;                        // exclusive prefix of list counts; pre[nl] = total
-    int* start = table + a.max_lists + 1;    // list start inside the row's list region
-    int* slot_pos = start + a.max_lists;     // per slot: first position of its segment
-    int* slot_len = slot_pos + a.max_slots;  // per slot: capacity of each warp's list
+    int* pre = table;                      // exclusive prefix of list counts; pre[nl] = total
+    int* start = table + a.max_lists + 1;  // list start inside the row's list region
 
     // ---- list table of the row
     float m_all = -kInf;
@@ -94,37 +92,47 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
         const int c_first = cta_of_tile(x0, T, a.C);
         const int slots = cta_of_tile(x0 + g.tiles - 1, T, a.C) - c_first + 1;
         nl = slots * g.WPK;  // <= max_lists (checked by the host)
-        // the first list's count and maximum are requested before the slot
-        // table is built, so their latency overlaps it
+        // Each thread owns a run of consecutive lists: it requests their counts
+        // and maxima all at once, works out where each list starts (the
+        // streaming CTA's segment of the row, split evenly over its warps)
+        // while they are in flight, and keeps the clamped counts for the scan.
         const size_t rbase = static_cast<size_t>(row) * g.S_cap * g.WPK;
-        const int cu_first = tid < nl ? a.seg_cnt[rbase + tid] : 0;
-        const float mall_first = tid < nl ? a.seg_mall[rbase + tid] : -kInf;
-        // per-slot position offset and tile count of the streaming CTA's segment
-        for (int sl = tid; sl < slots; sl += kThreads) {
-            const int c = c_first + sl;
-            const long long t0 = cta_tile_begin(T, a.C, c), t1 = cta_tile_begin(T, a.C, c + 1);
-            const long long s0 = t0 > x0 ? t0 : x0;
-            const long long s1 = t1 < x0 + g.tiles ? t1 : x0 + g.tiles;
-            slot_pos[sl] = static_cast<int>((s0 - x0) * g.P);
-            slot_len[sl] = static_cast<int>((s1 - s0) * g.MBW * 16);  // entries a warp can hold
-        }
-        __syncthreads();
-        // counts (coalesced reads), clamped to each list's capacity
-        float mloc = -kInf;
-        for (int j = tid; j < nl; j += kThreads) {
-            const int cu = j == tid ? cu_first : a.seg_cnt[rbase + j];
-            const int sl = j / g.WPK;
-            const int cap = slot_len[sl];
-            start[j] = slot_pos[sl] + (j - sl * g.WPK) * cap;
-            pre[j] = cu < 0 ? 0 : (cu > cap ? cap : cu);
-            mloc = fmaxf(mloc, j == tid ? mall_first : a.seg_mall[rbase + j]);
-        }
-        __syncthreads();
-        // exclusive scan: each thread owns a run of consecutive lists
         const int per = (nl + kThreads - 1) / kThreads;
         const int j0 = min(nl, tid * per), j1 = min(nl, j0 + per);
+        float mloc = -kInf;
         int run = 0;
-        for (int j = j0; j < j1; ++j) run += pre[j];
+        constexpr int kRun = 4;  // counts in flight per thread
+        for (int jb = j0; jb < j1; jb += kRun) {
+            int cu[kRun];
+            float mm[kRun];
+#pragma unroll
+            for (int u = 0; u < kRun; ++u) {
+                cu[u] = jb + u < j1 ? a.seg_cnt[rbase + jb + u] : 0;
+                mm[u] = jb + u < j1 ? a.seg_mall[rbase + jb + u] : -kInf;
+            }
+            int sl_prev = -1, pos = 0, cap = 0;
+#pragma unroll
+            for (int u = 0; u < kRun; ++u) {
+                const int j = jb + u;
+                if (j < j1) {
+                    const int sl = j / g.WPK;
+                    if (sl != sl_prev) {
+                        const int c = c_first + sl;
+                        const long long t0 = cta_tile_begin(T, a.C, c), t1 = cta_tile_begin(T, a.C, c + 1);
+                        const long long s0 = t0 > x0 ? t0 : x0;
+                        const long long s1 = t1 < x0 + g.tiles ? t1 : x0 + g.tiles;
+                        pos = static_cast<int>((s0 - x0) * g.P);
+                        cap = static_cast<int>((s1 - s0) * g.MBW * 16);  // entries a warp can hold
+                        sl_prev = sl;
+                    }
+                    start[j] = pos + (j - sl * g.WPK) * cap;
+                    const int cnt_j = cu[u] < 0 ? 0 : (cu[u] > cap ? cap : cu[u]);
+                    pre[j] = cnt_j;
+                    run += cnt_j;
+                    mloc = fmaxf(mloc, mm[u]);
+                }
+            }
+        }
         int inc = run;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -295,8 +303,8 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
 
 }  // namespace
 
-size_t gather_smem_bytes(int max_lists, int max_slots) {
-    return (2 * static_cast<size_t>(max_lists) + 1 + 2 * static_cast<size_t>(max_slots)) * sizeof(int);
+size_t gather_smem_bytes(int max_lists) {
+    return (2 * static_cast<size_t>(max_lists) + 1) * sizeof(int);
 }
 
 // Lets both block orders of one instantiation use the list table's
@@ -316,7 +324,7 @@ cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     const dim3 grid = a.part_major ? dim3(static_cast<unsigned>(rows), static_cast<unsigned>(a.parts))
                                    : dim3(static_cast<unsigned>(a.parts), static_cast<unsigned>(rows));
-    const size_t smem = gather_smem_bytes(a.max_lists, a.max_slots);
+    const size_t smem = gather_smem_bytes(a.max_lists);
     if (smem > static_cast<size_t>(kGatherMaxSmem) || a.cmb.parts != a.parts) return cudaErrorInvalidValue;
 #define SAGA_GATHER_CASE(D_, DK_, NT_)                                                         \
     if (a.g.dv == D_ && a.g.d == DK_ && a.g.NT == NT_) {                                       \

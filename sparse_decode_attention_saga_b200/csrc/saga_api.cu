@@ -378,7 +378,6 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         ga.parts = gather_parts(g, dev);
         ga.part_major = ga.parts >= kPartMajorParts;
         ga.max_lists = 1;
-        ga.max_slots = 1;
         ga.v = v;
         ga.idx = sa.idx;
         ga.list_s = sa.s;
@@ -399,7 +398,7 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     // fused: stream K, compare on chip, lists -> gathered PV with the row merge
     const int C = stream_ctas(g, dev, stream_shape(g).ctas_per_sm);
     const int slots = max_slots(g, static_cast<long long>(g.b) * g.tiles, C);
-    if (gather_smem_bytes(slots * g.WPK, slots) > static_cast<size_t>(kGatherMaxSmem))
+    if (gather_smem_bytes(slots * g.WPK) > static_cast<size_t>(kGatherMaxSmem))
         return SAGA_ERR_UNSUPPORTED;  // checked before anything is enqueued
     CUtensorMap kmap;
     if ((st = encode_cache_map(&kmap, k, g, g.hk, g.d))) return st;
@@ -425,7 +424,6 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     ga.C = a.C;
     ga.parts = gather_parts(g, dev);
     ga.part_major = ga.parts >= kPartMajorParts;
-    ga.max_slots = slots;
     ga.max_lists = slots * g.WPK;
     ga.v = v;
     ga.seg_list = a.list;

@@ -126,7 +126,6 @@ struct GatherArgs {
     int part_major; // grid (rows, parts) instead of (parts, rows)
     int C;          // kListSegments: grid of the fused kernel
     int max_lists;  // lists per row at most (kListSegments: slots * WPK; else 1)
-    int max_slots;  // kListSegments: streaming-CTA slots per row at most; else 1
     const void* v;
     const int32_t* idx;       // kListContiguous: positions [rows][l]
     const int32_t* cnt;       // kListContiguous: counts [rows]
@@ -141,7 +140,7 @@ struct GatherArgs {
     uint32_t* tickets;
     CombineArgs cmb;
 };
-size_t gather_smem_bytes(int max_lists, int max_slots);
+size_t gather_smem_bytes(int max_lists);
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream);
 
 // Dense flash-decoding kernel (K and V streamed) -> partial records.
