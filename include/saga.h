@@ -123,8 +123,15 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
  *   out[b,i,:] = sum_kept softmax(s) V[b,j,vh(i),:].
  * The min() keeps the row's maximal entries when a stale threshold lies
  * above every logit (the pages are silent on that case).
- *   logits_in != NULL: the logits are read from there (q, k unused); the
- *                      select/compact, gathered-PV and combine kernels run.
+ *   logits_in != NULL: the logits are read from there (q, k may be NULL);
+ *                      the select/compact, gathered-PV and combine kernels
+ *                      run.  Exception: with sel_idx == NULL, q and k given,
+ *                      and few long rows (b*h_q <= 64 and l_kv >= 65536,
+ *                      where one compare CTA per row would leave most of the
+ *                      GPU idle), the fused path below runs instead; it
+ *                      recomputes the same logits bit for bit with the same
+ *                      tensor-core routine as saga_topn_refresh, so the kept
+ *                      set is identical.
  *   logits_in == NULL and sel_idx == NULL: the fused kernel computes the
  *                      logits on chip, compares, and gathers only the kept
  *                      value rows; logits never reach device memory.

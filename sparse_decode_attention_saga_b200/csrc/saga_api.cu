@@ -198,6 +198,10 @@ int stream_ctas(const Geometry& g, const DeviceInfo& dev, int per_sm) {
 // (measured: Llama-shaped batch 1 at 8K, 23.5 -> 21.5 us per reuse step;
 // row-major stays faster at batch 16, 233 -> 229 us).
 constexpr int kPartMajorParts = 16;
+// A decode step given stored logits streams K instead when it has at most
+// this many rows of at least this many positions.
+constexpr long long kFusedFewRows = 64;
+constexpr int kFusedMinPositions = 65536;
 
 int gather_parts(const Geometry& g, const DeviceInfo& dev) {
     const long long rows = static_cast<long long>(g.b) * g.hq;
@@ -350,6 +354,14 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     uint32_t* err = ws_at<uint32_t>(ws, L.err);
     const long long rows = static_cast<long long>(g.b) * g.hq;
     float* records = ws_at<float>(ws, L.records);
+    // Few long rows: the compare kernel's one CTA per row leaves most SMs
+    // idle (Llama-shaped batch 1 at 128K: refresh step 110 us over stored
+    // logits, 89 us when the decode streams K again through the fused path,
+    // which yields the same logits bit for bit; at 8K to 32K the stored
+    // logits stay faster).
+    if (logits_in && !sel_idx && rows <= kFusedFewRows && g.l >= kFusedMinPositions && q && k &&
+        aligned(q, 16) && aligned(k, 16))
+        logits_in = nullptr;
 
     if (logits_in || sel_idx) {
         // stored logits -> compare/compact -> gathered PV -> combine
