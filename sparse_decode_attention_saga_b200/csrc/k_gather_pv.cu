@@ -36,7 +36,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMinShare = 128;  // kept entries per CTA at least
 #ifndef SAGA_GATHER_INFLIGHT
-#define SAGA_GATHER_INFLIGHT 4
+#define SAGA_GATHER_INFLIGHT 2
 #endif
 #ifndef SAGA_GATHER_MINBLOCKS
 #define SAGA_GATHER_MINBLOCKS 4
