@@ -313,7 +313,9 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
         g_launches += 1;
         return cuda_status(launch_fill(thresh_out, rows, -std::numeric_limits<float>::infinity(), s));
     }
-    cudaError_t e = cudaMemsetAsync(ws_at<uint8_t>(ws, L.hist), 0, L.cnt - L.hist, s);
+    // tickets (a safety net: they are kept at zero between launches),
+    // histograms and radix state
+    cudaError_t e = cudaMemsetAsync(ws_at<uint8_t>(ws, L.tickets), 0, L.cnt - L.tickets, s);
     if (e != cudaSuccess) return SAGA_ERR_CUDA;
     RadixArgs r{};
     r.logits = logits;

@@ -66,15 +66,19 @@ SAGA_HD int slots_of_batch(int bb, int tiles, long long T, int C) {
     return cta_of_tile(x0 + tiles - 1, T, C) - cta_of_tile(x0, T, C) + 1;
 }
 
+// The regions up to `rowmax` depend only on the batch and head counts, so
+// their offsets do not move when the cached length changes (decode with a
+// growing cache); the per-row tickets, which must be zero on entry, live
+// there.
 struct WsLayout {
     size_t err;       // uint32 sticky flag (256-byte header)
-    size_t records;   // float [b*hq][S_cap * WPK][rec]
+    size_t tickets;   // uint32 [b*hq]  last-CTA tickets (zero on entry, left at zero)
     size_t hist;      // uint32 [kRadixPasses][b*hq][kRadixBins]
     size_t state;     // uint32 [b*hq][2]  (prefix, rank)
-    size_t tickets;   // uint32 [b*hq]
     size_t cnt;       // int32  [b*hq]
     size_t cand_cnt;  // int32  [b*hq][kRadixMaxChunks]  radix pass-1 candidates per chunk
     size_t rowmax;    // float  [b*hq]
+    size_t records;   // float  [b*hq][S_cap * WPK][rec]
     size_t seg_cnt;   // int32  [b*hq][S_cap][WPK]
     size_t seg_mall;  // float  [b*hq][S_cap][WPK]
     size_t list_idx;  // int32  [b*hq][l_pad]; with list_s also the int2 [b*hq][l_pad]
@@ -95,13 +99,13 @@ inline WsLayout workspace_layout(const Geometry& g) {
         return at;
     };
     w.err = take(256);
-    w.records = take(rows * g.S_cap * g.WPK * g.rec * sizeof(float));
+    w.tickets = take(rows * sizeof(uint32_t));
     w.hist = take(static_cast<size_t>(kRadixPasses) * rows * kRadixBins * sizeof(uint32_t));
     w.state = take(rows * 2 * sizeof(uint32_t));
-    w.tickets = take(rows * sizeof(uint32_t));
     w.cnt = take(rows * sizeof(int32_t));
     w.cand_cnt = take(rows * kRadixMaxChunks * sizeof(int32_t));
     w.rowmax = take(rows * sizeof(float));
+    w.records = take(rows * g.S_cap * g.WPK * g.rec * sizeof(float));
     w.seg_cnt = take(rows * g.S_cap * g.WPK * sizeof(int32_t));
     w.seg_mall = take(rows * g.S_cap * g.WPK * sizeof(float));
     w.list_idx = take(rows * g.l_pad * sizeof(int32_t));
