@@ -60,6 +60,10 @@ def _growth_loop(w: Workload, seed: int):
     ("llama_like", 2, 32, 4, 8, 64, 700, 20, 4, 9),
     ("qwen_like", 1, 12, 1, 2, 128, 1023, 30, 3, 8),
     ("tile_boundary", 2, 8, 2, 4, 64, 254, 8, 4, 6),  # grows across a tile edge (128-position tiles)
+    # 32-position tiles and one refresh: the reuse steps that follow see the
+    # tile count (and the workspace's record region) grow without a refresh
+    # clearing anything in between
+    ("small_tiles_one_refresh", 2, 8, 8, 8, 64, 94, 10, 16, 9),
 ], ids=lambda s: s[0])
 def test_decode_with_cache_growth_matches_oracle(shape):
     name, b, hq, hk, hv, d, l0, N, n, steps = shape
