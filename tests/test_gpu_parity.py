@@ -261,7 +261,7 @@ def test_resume_from_saved_state_is_bit_identical():
 # ---------------------------------------------------------------- full-size workloads
 
 FULL = ["qwen_b1_32k", "llama_b16_128k", "qwen_b16_128k_saga_N1024", "qwen_b16_128k_gqa_N2048",
-        "llama_sweep_b1_l128k", "llama_sweep_b16_l8k"]
+        "llama_sweep_b1_l128k", "llama_sweep_b16_l8k", "sigma_b16_128k"]
 
 
 @pytest.mark.parametrize("name", FULL)
