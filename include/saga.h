@@ -144,6 +144,61 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
                       int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
                       saga_stream_t stream);
 
+/* ---- Sequence shards (the pages run one GPU; this is an extension) ----
+ * A decode whose cached sequence is split into contiguous shards, one per
+ * rank (each rank's dims: its own l_kv and l_cap; the same b, heads and q).
+ * The threshold stays the exact N-th largest logit of the whole row: each
+ * rank histograms a digit of its own logits, the caller sums the histograms
+ * across ranks (an all-reduce), and every rank takes the same digit from the
+ * sum (3 passes: 11, 11 and 10 bits of an order-preserving key, as
+ * saga_topn_refresh).  Each rank then decodes its shard into a partial
+ * record per row, the caller gathers the records of all ranks, and
+ * saga_merge_partials merges them (log-sum-exp) into the output a single
+ * GPU would give, empty-set rule included.  Callers order the calls of one
+ * rank on one stream; the cross-rank exchange is the caller's (NCCL). */
+
+/* Logits of this shard: logits_out[b,i,j] = q[b,i,:].k[b,j,kh(i),:]/sqrt(d),
+ * fp32, j < l_kv (the same values saga_topn_refresh computes). */
+int saga_qk_logits(const saga_dims* dims, const void* q, const void* k, float* logits_out,
+                   void* ws, size_t ws_bytes, saga_stream_t stream);
+
+/* Digit histogram of radix pass `pass` (0, 1, 2) over this shard's logits
+ * [b,h_q,l_kv]: hist[b*h_q][2048] (overwritten) counts, per row, the keys
+ * that carry the prefix in state[row] (ignored for pass 0) by their digit.
+ * state [b*h_q][2] uint32 is the one saga_topn_select_digit keeps. */
+int saga_topn_histogram(const saga_dims* dims, int32_t pass, const float* logits,
+                        const uint32_t* state, uint32_t* hist, saga_stream_t stream);
+
+/* Digit choice of pass `pass` from the histograms summed over every shard:
+ * updates state [b*h_q][2] (prefix, remaining rank; rank 0 once the row's
+ * threshold is known) and, once known, thresh_out[b*h_q]: the N-th largest
+ * logit of the whole row, or -inf when N is at least the row's total
+ * length (decided in pass 0).  Identical sums give identical results on
+ * every rank. */
+int saga_topn_select_digit(const saga_dims* dims, int32_t N, int32_t pass, const uint32_t* hist,
+                           uint32_t* state, float* thresh_out, saga_stream_t stream);
+
+/* saga_atopn_decode over this shard, without normalising: part[b*h_q] gets
+ * records of d_v + 4 floats (m, l, count, row max, o[d_v]):
+ *   count > 0: m = the shard's largest logit (kept), l = sum exp(s - m) and
+ *              o = sum exp(s - m) V over the shard's kept entries;
+ *   count = 0: m = -inf, l = number of the shard's positions at its row max,
+ *              o = the sum of their value rows (the empty-set rule's data).
+ * count is stored as int32 bits.  q and k are required even with logits_in
+ * (a shard that keeps nothing recomputes its maxima from them). */
+int saga_atopn_decode_partial(const saga_dims* dims, const void* q, const void* k, const void* v,
+                              const float* thresh, const float* logits_in, float* part, void* ws,
+                              size_t ws_bytes, saga_stream_t stream);
+
+/* out[b*h_q][d_v] from the R shards' records parts[R][b*h_q][d_v + 4]:
+ * with M the largest m over records that kept something,
+ * out = sum_r exp(m_r - M) o_r / sum_r exp(m_r - M) l_r; when no shard kept
+ * anything, the mean of the value rows at the row's maximum over the shards
+ * holding it.  sel_cnt (nullable): kept entries per row (or the number at
+ * the maximum).  Only b, h_q and the value head dim of dims are used. */
+int saga_merge_partials(const saga_dims* dims, const float* parts, int32_t R, float* out,
+                        int32_t* sel_cnt, saga_stream_t stream);
+
 /* Allocation-free threshold refresh (the paper has no counterpart; this is
  * a convenience of this library).  Computes exactly what saga_topn_refresh
  * computes with logits_in != NULL -- thresh_out[b,i] = the N-th largest of

@@ -27,7 +27,8 @@ EXPORTS = (
     "saga_workspace_bytes", "saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
     "saga_workspace_reset", "saga_workspace_error", "saga_status_string", "saga_launch_count",
     "saga_set_kernel_events", "saga_version", "saga_topn_refresh_noalloc",
-    "saga_selftest_wait_timeout", "saga_cache_append",
+    "saga_selftest_wait_timeout", "saga_cache_append", "saga_qk_logits", "saga_topn_histogram",
+    "saga_topn_select_digit", "saga_atopn_decode_partial", "saga_merge_partials",
 )
 
 
@@ -78,8 +79,15 @@ def load(path: str | None = None):
         lib.saga_launch_count.restype = ctypes.c_uint64
         lib.saga_set_kernel_events.argtypes = [P, P]
         lib.saga_set_kernel_events.restype = None
+        lib.saga_qk_logits.argtypes = [D, P, P, P, P, SZ, P]
+        lib.saga_topn_histogram.argtypes = [D, I32, P, P, P, P]
+        lib.saga_topn_select_digit.argtypes = [D, I32, I32, P, P, P, P]
+        lib.saga_atopn_decode_partial.argtypes = [D, P, P, P, P, P, P, P, SZ, P]
+        lib.saga_merge_partials.argtypes = [D, P, I32, P, P, P]
         for f in ("saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
-                  "saga_workspace_reset", "saga_workspace_error", "saga_version"):
+                  "saga_workspace_reset", "saga_workspace_error", "saga_version", "saga_qk_logits",
+                  "saga_topn_histogram", "saga_topn_select_digit", "saga_atopn_decode_partial",
+                  "saga_merge_partials"):
             getattr(lib, f).restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -154,6 +162,39 @@ def cache_append(d, k_new, v_new, k, v, stream=None) -> None:
     _check("saga_cache_append",
            load().saga_cache_append(ctypes.byref(d), _ptr(k_new), _ptr(v_new), _ptr(k), _ptr(v),
                                     _stream(stream)))
+
+
+# ---- sequence shards (one rank's calls; the cross-rank sums are the caller's)
+
+def qk_logits(d, q, k, logits_out, ws, stream=None) -> None:
+    _check("saga_qk_logits",
+           load().saga_qk_logits(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(logits_out), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def topn_histogram(d, pass_: int, logits, state, hist, stream=None) -> None:
+    _check("saga_topn_histogram",
+           load().saga_topn_histogram(ctypes.byref(d), int(pass_), _ptr(logits), _ptr(state),
+                                      _ptr(hist), _stream(stream)))
+
+
+def topn_select_digit(d, N: int, pass_: int, hist, state, thresh_out, stream=None) -> None:
+    _check("saga_topn_select_digit",
+           load().saga_topn_select_digit(ctypes.byref(d), int(N), int(pass_), _ptr(hist),
+                                         _ptr(state), _ptr(thresh_out), _stream(stream)))
+
+
+def atopn_decode_partial(d, q, k, v, thresh, logits_in, part, ws, stream=None) -> None:
+    _check("saga_atopn_decode_partial",
+           load().saga_atopn_decode_partial(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(thresh), _ptr(logits_in), _ptr(part), _ptr(ws),
+                                            ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def merge_partials(d, parts, R: int, out, sel_cnt=None, stream=None) -> None:
+    _check("saga_merge_partials",
+           load().saga_merge_partials(ctypes.byref(d), _ptr(parts), int(R), _ptr(out),
+                                      _ptr(sel_cnt), _stream(stream)))
 
 
 def selftest_wait_timeout(ws, limit_us: int, stream=None) -> None:

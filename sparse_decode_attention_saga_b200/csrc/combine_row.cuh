@@ -23,9 +23,11 @@ namespace saga {
 
 constexpr int kCombineThreads = 256;
 
+// raw: out_row gets the sum of the value rows at m_star instead of their
+// mean.  Returns their number (all lanes).
 template <int DV, int D, int NT>  // D: key/query head dim, DV: value head dim
-__device__ void fallback_row(const CombineArgs& a, long long row, float m_star, float* out_row,
-                             int32_t* cnt_out, uint8_t* kbuf) {
+__device__ int fallback_row(const CombineArgs& a, long long row, float m_star, float* out_row,
+                            int32_t* cnt_out, uint8_t* kbuf, bool raw = false) {
     const Geometry& g = a.g;
     const int lane = threadIdx.x & 31;
     const int bb = static_cast<int>(row / g.hq);
@@ -85,8 +87,9 @@ __device__ void fallback_row(const CombineArgs& a, long long row, float m_star, 
         }
     }
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) out_row[lane * CPL + c] = osum[c] / static_cast<float>(count);
+    for (int c = 0; c < CPL; ++c) out_row[lane * CPL + c] = raw ? osum[c] : osum[c] / static_cast<float>(count);
     if (lane == 0 && cnt_out) *cnt_out = count;
+    return count;
 }
 
 // Number of partial records of row (of batch element bb).
@@ -275,25 +278,50 @@ __device__ void merge_same_reference(const CombineArgs& a, long long row, int R,
         lsum += red_l[w];
         cnt += red_c[w];
     }
-    float* out_row = a.out + static_cast<size_t>(row) * D;
+    float* part = a.part ? a.part + static_cast<size_t>(row) * (D + kRecHeader) : nullptr;
+    float* out_row = part ? part + kRecHeader : a.out + static_cast<size_t>(row) * D;
     if (cnt == 0) {
         if (a.fallback) {
-            if (warp == 0)
-                fallback_row<D, DK, NT>(a, row, m_all, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf);
+            if (warp == 0) {
+                const int c = fallback_row<D, DK, NT>(a, row, m_all, out_row,
+                                                      part || !a.sel_cnt ? nullptr : a.sel_cnt + row,
+                                                      kbuf, part != nullptr);
+                if (part && lane == 0) {
+                    part[0] = -kInf;
+                    part[1] = static_cast<float>(c);
+                    part[2] = __int_as_float(0);
+                    part[3] = m_all;
+                }
+            }
         } else {
             for (int k = tid; k < D; k += kCombineThreads) out_row[k] = 0.f;
-            if (tid == 0 && a.sel_cnt) a.sel_cnt[row] = 0;
+            if (tid == 0 && part) {
+                part[0] = -kInf;
+                part[1] = 0.f;
+                part[2] = __int_as_float(0);
+                part[3] = m_all;
+            }
+            if (tid == 0 && !part && a.sel_cnt) a.sel_cnt[row] = 0;
         }
         return;
     }
-    const float inv = 1.f / lsum;
+    const float inv = part ? 1.f : 1.f / lsum;
     for (int k = tid; k < D; k += kCombineThreads) {
         float v = 0.f;
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) v += red_o[w][k];
         out_row[k] = v * inv;
     }
-    if (tid == 0 && a.sel_cnt) a.sel_cnt[row] = cnt;
+    if (tid == 0) {
+        if (part) {
+            part[0] = m_all;  // every share was weighted with exp(s - m_all)
+            part[1] = lsum;
+            part[2] = __int_as_float(cnt);
+            part[3] = m_all;
+        } else if (a.sel_cnt) {
+            a.sel_cnt[row] = cnt;
+        }
+    }
 }
 
 }  // namespace saga

@@ -15,7 +15,8 @@
 // logit, for the gather kernel) is written at its rank, so the output is
 // ascending.  The row's largest logit is stored for the gather kernel's
 // softmax.  If nothing passed (only possible when tau > row max) the row is
-// compacted again against its max.
+// compacted again against its max, unless keep_max is 0 (a sequence shard,
+// whose empty-set rule belongs to the whole row).
 #include "saga_device.cuh"
 #include "saga_kernels.h"
 
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
             }
             __syncthreads();
         }
-        if (total > 0) break;
+        if (total > 0 || !a.keep_max) break;
     }
     if (tid == 0) a.cnt[row] = total;
 }

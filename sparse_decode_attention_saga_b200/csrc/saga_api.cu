@@ -336,13 +336,17 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
     return cuda_status(launch_radix_select(r, s));
 }
 
-int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const void* v,
-                      const float* thresh, const float* logits_in, float* out, int32_t* sel_idx,
-                      int32_t* sel_cnt, void* ws, size_t ws_bytes, saga_stream_t stream) {
+// One decode step; the merged rows go to out (normalised), or with part to
+// part as unnormalised per-row records (a sequence shard's contribution).
+static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k, const void* v,
+                             const float* thresh, const float* logits_in, float* out, float* part,
+                             int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
+                             saga_stream_t stream) {
     Geometry g;
     int st = make_geometry(dims, &g);
     if (st) return st;
-    if (!v || !aligned(v, 16) || !thresh || !aligned(thresh, 4) || !out || !aligned(out, 4))
+    if (!v || !aligned(v, 16) || !thresh || !aligned(thresh, 4) ||
+        (out ? !aligned(out, 4) : (!part || !aligned(part, 4))))
         return SAGA_ERR_INVALID_ARG;
     if (logits_in ? !aligned(logits_in, 4) : (!q || !k || !aligned(q, 16) || !aligned(k, 16)))
         return SAGA_ERR_INVALID_ARG;
@@ -382,6 +386,9 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         sa.s = ws_at<float>(ws, L.list_s);
         sa.cnt = ws_at<int32_t>(ws, L.cnt);
         sa.rowmax = ws_at<float>(ws, L.rowmax);
+        // a shard keeps nothing when nothing passes: the whole row's maxima
+        // are found when the shards' records are merged
+        sa.keep_max = part ? 0 : 1;
         cudaError_t e = launch_select_compact(sa, s);
         g_launches += 1;
         if (e != cudaSuccess) return SAGA_ERR_CUDA;
@@ -404,7 +411,14 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
         ga.cmb.parts = ga.parts;
         ga.cmb.records = records;
         ga.cmb.out = out;
+        ga.cmb.part = part;
         ga.cmb.sel_cnt = sel_cnt;
+        if (part) {  // a shard that kept nothing reports its maxima (recomputed from q and k)
+            ga.cmb.fallback = 1;
+            ga.cmb.q = q;
+            ga.cmb.k = k;
+            ga.cmb.v = v;
+        }
         g_launches += 1;
         return cuda_status(launch_gather_pv(ga, s));
     }
@@ -454,9 +468,104 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     ga.cmb.v = v;
     ga.cmb.records = records;
     ga.cmb.out = out;
+    ga.cmb.part = part;
     ga.cmb.sel_cnt = sel_cnt;
     g_launches += 1;
     return cuda_status(launch_gather_pv(ga, s));
+}
+
+int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const void* v,
+                      const float* thresh, const float* logits_in, float* out, int32_t* sel_idx,
+                      int32_t* sel_cnt, void* ws, size_t ws_bytes, saga_stream_t stream) {
+    if (!out) return SAGA_ERR_INVALID_ARG;
+    return atopn_decode_impl(dims, q, k, v, thresh, logits_in, out, nullptr, sel_idx, sel_cnt, ws,
+                             ws_bytes, stream);
+}
+
+int saga_atopn_decode_partial(const saga_dims* dims, const void* q, const void* k, const void* v,
+                              const float* thresh, const float* logits_in, float* part, void* ws,
+                              size_t ws_bytes, saga_stream_t stream) {
+    // q and k are needed even with stored logits: a shard that keeps nothing
+    // recomputes its row maxima from them
+    if (!part || !q || !k || !aligned(q, 16) || !aligned(k, 16)) return SAGA_ERR_INVALID_ARG;
+    return atopn_decode_impl(dims, q, k, v, thresh, logits_in, nullptr, part, nullptr, nullptr, ws,
+                             ws_bytes, stream);
+}
+
+int saga_merge_partials(const saga_dims* dims, const float* parts, int32_t R, float* out,
+                        int32_t* sel_cnt, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (R <= 0 || !parts || !aligned(parts, 4) || !out || !aligned(out, 4) ||
+        (sel_cnt && !aligned(sel_cnt, 4)))
+        return SAGA_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    MergeArgs a{};
+    a.parts = parts;
+    a.R = R;
+    a.rows = static_cast<long long>(g.b) * g.hq;
+    a.out = out;
+    a.sel_cnt = sel_cnt;
+    g_launches += 1;
+    return cuda_status(launch_merge_parts(g.dv, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int saga_qk_logits(const saga_dims* dims, const void* q, const void* k, float* logits_out, void* ws,
+                   size_t ws_bytes, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (!q || !k || !logits_out || !aligned(q, 16) || !aligned(k, 16) || !aligned(logits_out, 4))
+        return SAGA_ERR_INVALID_ARG;
+    if ((st = check_ws(g, ws, ws_bytes))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    const WsLayout L = workspace_layout(g);
+    return run_logits(g, dev, q, k, logits_out, ws_at<uint32_t>(ws, L.err),
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int saga_topn_histogram(const saga_dims* dims, int32_t pass, const float* logits,
+                        const uint32_t* state, uint32_t* hist, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (pass < 0 || pass >= kRadixPasses || !logits || !aligned(logits, 4) || !hist ||
+        !aligned(hist, 4) || (pass > 0 && (!state || !aligned(state, 4))))
+        return SAGA_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    ShardHistArgs a{};
+    a.logits = logits;
+    a.rows = static_cast<long long>(g.b) * g.hq;
+    a.l = g.l;
+    a.chunks = radix_chunks(a.rows, g.l, dev.sms);
+    a.state = state;
+    a.hist = hist;
+    g_launches += 1;
+    return cuda_status(launch_shard_hist(pass, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int saga_topn_select_digit(const saga_dims* dims, int32_t N, int32_t pass, const uint32_t* hist,
+                           uint32_t* state, float* thresh_out, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (N <= 0 || pass < 0 || pass >= kRadixPasses || !hist || !aligned(hist, 4) || !state ||
+        !aligned(state, 4) || !thresh_out || !aligned(thresh_out, 4))
+        return SAGA_ERR_INVALID_ARG;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    ShardDigitArgs a{};
+    a.hist = hist;
+    a.rows = static_cast<long long>(g.b) * g.hq;
+    a.N = N;
+    a.state = state;
+    a.thresh = thresh_out;
+    g_launches += 1;
+    return cuda_status(launch_shard_digit(pass, a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const void* v,

@@ -89,6 +89,7 @@ struct SelectArgs {
     float* s;      // [rows][l]  their logits, same order
     int32_t* cnt;  // [rows]
     float* rowmax; // [rows]     largest logit of the row
+    int keep_max;  // nothing passed: keep the row's maxima (1) or nothing (0)
 };
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream);
 
@@ -113,6 +114,11 @@ struct CombineArgs {
     const float* records;
     float* out;
     int32_t* sel_cnt;
+    // Optional, for a sequence shard: the row's merged but unnormalised
+    // record (m, l, count, row max, o[dv]) goes to part[row] instead of out
+    // (count 0: m = -inf, l = number of positions at the row max, o = the
+    // sum of their value rows).
+    float* part;
 };
 // Gathered softmax-PV over kept lists -> partial records.
 enum ListMode : int {
@@ -161,6 +167,35 @@ cudaError_t launch_dense(const CUtensorMap& kmap, const CUtensorMap& vmap, const
                          cudaStream_t stream);
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t stream);
+
+// Sequence shards: digit histograms of this shard's logits (summed across
+// shards by the caller), the digit choice on the summed histograms, and the
+// merge of the shards' partial records.
+struct ShardHistArgs {
+    const float* logits;    // [rows][l] this shard's logits
+    long long rows;
+    int l;
+    int chunks;             // CTAs per row
+    const uint32_t* state;  // [rows][2] (prefix, rank) of the earlier passes
+    uint32_t* hist;         // [rows][kRadixBins] out (cleared first)
+};
+cudaError_t launch_shard_hist(int pass, const ShardHistArgs& a, cudaStream_t stream);
+struct ShardDigitArgs {
+    const uint32_t* hist;   // [rows][kRadixBins] summed over the shards
+    long long rows;
+    int N;
+    uint32_t* state;        // [rows][2] in/out; rank 0: threshold known
+    float* thresh;          // [rows] written once known
+};
+cudaError_t launch_shard_digit(int pass, const ShardDigitArgs& a, cudaStream_t stream);
+struct MergeArgs {
+    const float* parts;     // [R][rows][dv + kRecHeader]
+    int R;
+    long long rows;
+    float* out;             // [rows][dv]
+    int32_t* sel_cnt;       // [rows] or null
+};
+cudaError_t launch_merge_parts(int dv, const MergeArgs& a, cudaStream_t stream);
 
 // Cache growth: new rows k_new [b,h_k,d], v_new [b,h_v,d] -> row `pos` of
 // k [b,l_cap,h_k,d] and v [b,l_cap,h_v,d].
