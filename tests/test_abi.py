@@ -154,3 +154,36 @@ def test_cache_append_validation(lib):
 def test_value_head_dim_validation(lib, hk, d, dv, ok):
     dims = _lib.dims(1, 16, hk, 8, d, 256, None, dv)
     assert (_lib.workspace_bytes(dims, 8) > 0) == ok
+
+
+def test_sequence_shard_call_validation(lib):
+    d = _lib.dims(1, 4, 1, 2, 64, 64)
+    need = _lib.workspace_bytes(d, 8)
+    big = _ws(need + 512)
+    base = (big.data_ptr() + 255) // 256 * 256
+    # radix pass out of range, missing state after pass 0, null histogram
+    assert lib.saga_topn_histogram(ctypes.byref(d), 3, 16, 16, 16, None) == _lib.SAGA_ERR_INVALID_ARG
+    assert lib.saga_topn_histogram(ctypes.byref(d), 1, 16, None, 16, None) == \
+        _lib.SAGA_ERR_INVALID_ARG
+    assert lib.saga_topn_histogram(ctypes.byref(d), 0, 16, None, None, None) == \
+        _lib.SAGA_ERR_INVALID_ARG
+    # N <= 0, pass out of range, null threshold output
+    assert lib.saga_topn_select_digit(ctypes.byref(d), 0, 0, 16, 16, 16, None) == \
+        _lib.SAGA_ERR_INVALID_ARG
+    assert lib.saga_topn_select_digit(ctypes.byref(d), 8, -1, 16, 16, 16, None) == \
+        _lib.SAGA_ERR_INVALID_ARG
+    assert lib.saga_topn_select_digit(ctypes.byref(d), 8, 2, 16, 16, None, None) == \
+        _lib.SAGA_ERR_INVALID_ARG
+    # the partial decode needs q and k even with stored logits, and a record buffer
+    assert lib.saga_atopn_decode_partial(ctypes.byref(d), None, None, 16, 16, 16, 16, base, need,
+                                         None) == _lib.SAGA_ERR_INVALID_ARG
+    assert lib.saga_atopn_decode_partial(ctypes.byref(d), 16, 16, 16, 16, None, None, base, need,
+                                         None) == _lib.SAGA_ERR_INVALID_ARG
+    # merge: at least one record set, aligned output
+    assert lib.saga_merge_partials(ctypes.byref(d), 16, 0, 16, None, None) == \
+        _lib.SAGA_ERR_INVALID_ARG
+    assert lib.saga_merge_partials(ctypes.byref(d), 16, 2, 18, None, None) == \
+        _lib.SAGA_ERR_INVALID_ARG
+    # logits: workspace too small
+    assert lib.saga_qk_logits(ctypes.byref(d), 16, 16, 16, base, need - 1, None) == \
+        _lib.SAGA_ERR_WORKSPACE
