@@ -191,8 +191,6 @@ int stream_ctas(const Geometry& g, const DeviceInfo& dev, int per_sm) {
     return C;
 }
 
-// CTAs per row of the gather kernel: about 8 per SM over all rows, never more
-// than the partial-record slots of a row.
 // From this many CTAs per row (few rows) the gather grid is part-major: most
 // rows then need only some of their parts, and the needed ones go first
 // (measured: Llama-shaped batch 1 at 8K, 23.5 -> 21.5 us per reuse step;
@@ -203,6 +201,8 @@ constexpr int kPartMajorParts = 16;
 constexpr long long kFusedFewRows = 64;
 constexpr int kFusedMinPositions = 65536;
 
+// CTAs per row of the gather kernel: about 8 per SM over all rows, never more
+// than the partial-record slots of a row.
 int gather_parts(const Geometry& g, const DeviceInfo& dev) {
     const long long rows = static_cast<long long>(g.b) * g.hq;
     long long parts = (8ll * dev.sms + rows - 1) / rows;
