@@ -261,6 +261,9 @@ def run_ours(args, world, rank, local):
     qs = make_queries(w, seed, "cuda", steps=total_steps)
     dec = AtopNDecoder.for_workload(w)
     stream = torch.cuda.Stream()
+    # the inputs and the decoder's zeroed workspace were made on the default
+    # stream; everything below runs on `stream`
+    torch.cuda.synchronize()
     launches0 = _lib.launch_count()
 
     with torch.cuda.stream(stream):
@@ -385,6 +388,7 @@ def run_ours(args, world, rank, local):
         Kg, Vg = make_cache(wg, seed, "cuda")
         gdec = AtopNDecoder.for_workload(wg)
         gqa_out = torch.empty_like(gdec.out)
+        torch.cuda.synchronize()  # its cache and workspace come from the default stream
         us_dense_gqa = time_steps(lambda r: gdec.dense(qs[r % 4], Kg, Vg, out=gqa_out), 10)
         assert gdec.error() == _lib.SAGA_OK
         del Kg, Vg, gdec, gqa_out
@@ -481,6 +485,7 @@ def run_ours(args, world, rank, local):
     for rep in range(2):  # the first pass warms up
         gdec = AtopNDecoder(w.batch, w.h_q, w.h_k, w.h_v, w.head_dim, w.l_kv - G, w.N, w.n,
                             l_cap=w.l_kv, v_head_dim=w.dv)
+        torch.cuda.synchronize()  # rows and workspace come from the default stream
         g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             g0.record(stream)
