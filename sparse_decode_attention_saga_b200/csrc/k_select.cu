@@ -9,7 +9,10 @@
 //
 // One CTA of 256 threads per (batch, query head) row.  A round covers
 // 4 x 256 x VEC positions: each thread reads VEC consecutive logits per
-// sub-round (16-byte loads when rows are 16-byte aligned), counts its kept
+// sub-round (16-byte loads when rows are 16-byte aligned; VEC = 16 when the
+// rows are few, so that the few CTAs keep 64 KB of loads in flight between
+// the round's barriers, VEC = 4 otherwise, which keeps four CTAs per SM and
+// the whole grid in one wave), counts its kept
 // ones, the counts are prefix-summed inside the warp (shuffles) and across
 // the 8 warps x 4 sub-rounds (warp 0), and every kept position (and its
 // logit, for the gather kernel) is written at its rank, so the output is
@@ -56,11 +59,15 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
 #pragma unroll
             for (int k = 0; k < kSub; ++k) {
                 const int j = base + (k * kThreads + tid) * VEC;
-                if (VEC == 4 && j + VEC <= a.l) {
-                    const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
-                    const float xs[4] = {x.x, x.y, x.z, x.w};
+                if (VEC >= 4 && j + VEC <= a.l) {
 #pragma unroll
-                    for (int c = 0; c < VEC; ++c) v[k][c] = xs[c];
+                    for (int h = 0; h < VEC / 4; ++h) {
+                        const float4 x = __ldg(reinterpret_cast<const float4*>(src + j) + h);
+                        v[k][4 * h] = x.x;
+                        v[k][4 * h + 1] = x.y;
+                        v[k][4 * h + 2] = x.z;
+                        v[k][4 * h + 3] = x.w;
+                    }
                 } else {
 #pragma unroll
                     for (int c = 0; c < VEC; ++c) v[k][c] = j + c < a.l ? __ldg(src + j + c) : -kInf;
@@ -140,8 +147,9 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream) {
     const bool vec = (a.l % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.logits) & 15u) == 0);
     const dim3 grid(static_cast<unsigned>(a.rows)), block(kThreads);
-    return vec ? launch_dependent(select_compact_kernel<4>, grid, block, 0, stream, a)
-               : launch_dependent(select_compact_kernel<1>, grid, block, 0, stream, a);
+    if (!vec) return launch_dependent(select_compact_kernel<1>, grid, block, 0, stream, a);
+    return a.wide ? launch_dependent(select_compact_kernel<16>, grid, block, 0, stream, a)
+                  : launch_dependent(select_compact_kernel<4>, grid, block, 0, stream, a);
 }
 
 }  // namespace saga

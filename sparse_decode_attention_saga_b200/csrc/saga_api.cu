@@ -200,6 +200,13 @@ constexpr int kPartMajorParts = 16;
 // this many rows of at least this many positions.
 constexpr long long kFusedFewRows = 64;
 constexpr int kFusedMinPositions = 65536;
+// Up to this many rows per SM the compare/compact kernel reads 16 logits per
+// thread per sub-round (more bytes in flight per CTA; two CTAs per SM by its
+// registers), beyond it 4 (measured on refresh steps: Qwen-shaped batch 16
+// at 128K 265 -> 238 us, Sigma-style 271 -> 238 us, Qwen-shaped batch 1 at
+// 32K 42.1 -> 39.0 us; the Llama-shaped batch 16, 512 rows, 491 -> 501 us
+// in two waves, so it keeps 4).
+constexpr long long kSelectWideRowsPerSm = 2;
 
 // CTAs per row of the gather kernel: about 8 per SM over all rows, never more
 // than the partial-record slots of a row.
@@ -389,6 +396,8 @@ static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k
         // a shard keeps nothing when nothing passes: the whole row's maxima
         // are found when the shards' records are merged
         sa.keep_max = part ? 0 : 1;
+        // up to two CTAs per SM of the wide form (its registers) in one wave
+        sa.wide = rows <= kSelectWideRowsPerSm * dev.sms;
         cudaError_t e = launch_select_compact(sa, s);
         g_launches += 1;
         if (e != cudaSuccess) return SAGA_ERR_CUDA;

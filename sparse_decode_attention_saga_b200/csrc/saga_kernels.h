@@ -90,6 +90,7 @@ struct SelectArgs {
     int32_t* cnt;  // [rows]
     float* rowmax; // [rows]     largest logit of the row
     int keep_max;  // nothing passed: keep the row's maxima (1) or nothing (0)
+    int wide;      // few rows: 16 logits per thread per sub-round instead of 4
 };
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream);
 

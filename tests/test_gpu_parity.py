@@ -34,6 +34,9 @@ SHAPES = [
     ("saga_1_8", 2, 16, 1, 8, 64, 3000, None),
     # h_q > 32: the reuse step takes the list path (compare kernel, gather, combine)
     ("hq64_lists", 2, 64, 4, 8, 64, 1500, None),
+    # more rows than two per SM: the compare kernel's 4-wide form (the shapes
+    # above take its 16-wide form for few rows)
+    ("rows_320", 10, 32, 4, 8, 64, 1000, None),
 ]
 
 
