@@ -430,6 +430,7 @@ def run_ours(args, world, rank, local):
     small = w.batch * w.h_q * (w.head_dim * 2 + 4)            # q + tau
     kern_bytes = k_bytes + small + kept * 8                   # + kept (pos, logit) lists
     step_ideal = k_bytes + U * w.dv * 2 + w.batch * w.h_q * (w.head_dim * 2 + w.dv * 4 + 4)
+    refresh_ideal = step_ideal + 2 * w.batch * w.h_q * w.l_kv * 4   # + logits written and read once
     peak, peak_kind = peaks()
     achieved = kern_bytes / (kern_us * 1e-6) / 1e9
 
@@ -532,6 +533,13 @@ def run_ours(args, world, rank, local):
                           "ideal_bytes": step_ideal, "us": us_reuse,
                           "achieved": step_ideal / (us_reuse * 1e-6) / 1e9,
                           "frac": step_ideal / (us_reuse * 1e-6) / 1e9 / peak},
+        "refresh_roofline": {"what": "refresh step (logits to HBM, radix select, compare/compact, "
+                                     "gather with row merge) vs the reuse step's ideal bytes, and vs "
+                                     "those plus one write and one read of the logits",
+                             "ideal_bytes": step_ideal, "ideal_bytes_with_logits": refresh_ideal,
+                             "us": us_refresh,
+                             "frac": step_ideal / (us_refresh * 1e-6) / 1e9 / peak,
+                             "frac_with_logits": refresh_ideal / (us_refresh * 1e-6) / 1e9 / peak},
         "grow": {"us_per_step": grow_us[-1], "steps": G, "l_kv": [w.l_kv - G + 1, w.l_kv],
                  "what": "append this step's K/V rows, then the Atop-N step over the grown "
                          "cache (refresh every n), eager, CUDA events"},
