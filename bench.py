@@ -437,78 +437,43 @@ def run_ours(args, world, rank, local):
     # ---- end to end through the public API with host buffers
     q_host = qs.cpu().pin_memory()
     out_host = torch.empty((args.steps,) + tuple(dec.out.shape), dtype=torch.float32).pin_memory()
-    q_dev = torch.empty_like(qs[0])
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def e2e_step(k):  # this step's query in from pinned host memory, its output back out
-        t = args.warmup + k
-        q_dev.copy_(q_host[t], non_blocking=True)
-        o = dec.step(t, q_dev, K, V)
-        out_host[k].copy_(o, non_blocking=True)
 
     barrier(world)
     torch.cuda.synchronize()
     if not cold:
-        # launched like the timed loop above: one CUDA graph of the K steps,
-        # each with its own host-to-device copy of its query and
-        # device-to-host copy of its output.  The copies run on two copy
-        # streams into and out of double buffers, so step k's output copy
-        # and step k + 1's query copy overlap the kernels around them
-        # (query buffer k mod 2 is refilled once step k - 2 has run, output
-        # buffer k mod 2 is rewritten once its copy of step k - 2 is out).
-        h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
-        q_buf = [torch.empty_like(qs[0]) for _ in range(2)]
-        o_buf = [torch.empty_like(dec.out) for _ in range(2)]
-        done = [torch.cuda.Event() for _ in range(args.steps)]
-        q_in = [torch.cuda.Event() for _ in range(args.steps)]
-        o_out = [torch.cuda.Event() for _ in range(args.steps)]
-        torch.cuda.synchronize()
-        e2e_graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(e2e_graph, stream=stream):
-            h2d.wait_stream(stream)   # the copy streams join the capture
-            d2h.wait_stream(stream)
-            for k in range(args.steps):
-                t = args.warmup + k
-                with torch.cuda.stream(h2d):
-                    if k >= 2:
-                        h2d.wait_event(done[k - 2])
-                    q_buf[k % 2].copy_(q_host[t], non_blocking=True)
-                    q_in[k].record(h2d)
-                stream.wait_event(q_in[k])
-                if k >= 2:
-                    stream.wait_event(o_out[k - 2])
-                dec.step(t, q_buf[k % 2], K, V, out=o_buf[k % 2])
-                done[k].record(stream)
-                with torch.cuda.stream(d2h):
-                    d2h.wait_event(done[k])
-                    out_host[k].copy_(o_buf[k % 2], non_blocking=True)
-                    o_out[k].record(d2h)
-            stream.wait_stream(h2d)
-            stream.wait_stream(d2h)
-        with torch.cuda.stream(stream):
-            e2e_graph.replay()        # untimed: the first launch uploads the graph
+        # launched like the timed loop above: the K steps as one CUDA graph
+        # (AtopNDecoder.host_loop: each step's query copied in from pinned
+        # host memory and its output copied out, on two copy streams with
+        # double buffers, overlapping the neighbouring steps' kernels)
+        loop = dec.host_loop(K, V, q_host, out_host, args.warmup, args.steps, stream=stream)
+        loop.replay()             # untimed: the first launch uploads the graph
         stream.synchronize()
         with torch.cuda.stream(stream):
             e0.record(stream)
-            e2e_graph.replay()
+            loop.replay()
             e1.record(stream)
         stream.synchronize()
         e2e_ms = e0.elapsed_time(e1)
-        del e2e_graph
+        del loop
     else:
-        # cold like the timed loop above: one CUDA graph per step with its
-        # copies, L2 flushed before every step outside the events
-        e2e_graphs = [capture([lambda k=k: e2e_step(k)]) for k in range(args.steps)]
+        # cold like the timed loop above: one host loop of one step per step,
+        # L2 flushed before every step outside the events
+        loops = [dec.host_loop(K, V, q_host, out_host[k:k + 1], args.warmup + k, 1, stream=stream)
+                 for k in range(args.steps)]
+        for lp in loops:          # untimed first launches, in step order
+            lp.replay()
+        stream.synchronize()
         e2e_ms = 0.0
-        for g in e2e_graphs:
+        for lp in loops:
             with torch.cuda.stream(stream):
                 flush()
                 e0.record(stream)
-                g.replay()
+                lp.replay()
                 e1.record(stream)
             e1.synchronize()
             e2e_ms += e0.elapsed_time(e1)
-        del e2e_graphs
+        del loops
     barrier(world)
     e2e_us = max_over_ranks(e2e_ms * 1e3 / args.steps, world)
     # Each step's own output reached the host: the last two steps (one per
@@ -594,8 +559,8 @@ def run_ours(args, world, rank, local):
                 "timing": ("one CUDA-graph replay of the K steps, each with its own copies in "
                            "and out of pinned host memory on two copy streams (double buffers, "
                            "overlapping the neighbouring steps' kernels)") if not cold else
-                          "one CUDA graph per step with its copies, CUDA events around each "
-                          "replay, L2 flushed before each"},
+                          "one host loop (CUDA graph) per step with its copies, CUDA events "
+                          "around each replay, L2 flushed before each"},
         "clocks": sampler.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:

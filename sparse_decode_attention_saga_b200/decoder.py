@@ -6,6 +6,8 @@ refresh schedule of "More Value per Key" (ai.info summary, Key Contributions
 #2: exact top-N thresholds computed once every n tokens and reused between):
 step t refreshes when t mod n == 0, then decodes with the stored thresholds.
 Every step is two or three C calls; all compute runs in libsaga.so.
+``HostLoop`` (``AtopNDecoder.host_loop``) runs a span of steps as one CUDA
+graph fed from, and writing to, pinned host memory.
 """
 from __future__ import annotations
 
@@ -85,3 +87,66 @@ class AtopNDecoder:
 
     def error(self, stream=None) -> int:
         return _lib.workspace_error(self.ws, stream)
+
+    def host_loop(self, k, v, q_host, out_host, t0: int, steps: int, stream=None) -> "HostLoop":
+        """Captures decode steps t0 .. t0 + steps - 1 fed from pinned host
+        memory (see HostLoop); the decoder must have run a step outside a
+        capture first, and its cached length stays fixed inside the loop."""
+        return HostLoop(self, k, v, q_host, out_host, t0, steps, stream)
+
+
+class HostLoop:
+    """A decode loop whose queries come from, and whose outputs go to, pinned
+    host memory: step t copies q_host[t] in and its output out to
+    out_host[t - t0].  One CUDA graph holds all the steps; the copies run on
+    two copy streams into and out of double buffers, so that they overlap the
+    kernels of the neighbouring steps: query buffer t mod 2 is refilled once
+    step t - 2 has run, and output buffer t mod 2 is rewritten once its copy
+    of step t - 2 is out.  The graph keeps the addresses of k, v and the host
+    buffers; replay() enqueues the whole loop on the loop's stream."""
+
+    def __init__(self, dec, k, v, q_host, out_host, t0, steps, stream=None):
+        steps, t0 = int(steps), int(t0)
+        if steps < 1 or t0 < 0 or q_host.shape[0] < t0 + steps or out_host.shape[0] < steps:
+            raise ValueError("host buffers do not cover the steps")
+        if not (q_host.is_pinned() and out_host.is_pinned()):
+            raise ValueError("host buffers must be pinned")
+        self.stream = torch.cuda.Stream() if stream is None else stream
+        self.q_host, self.out_host = q_host, out_host
+        self._h2d, self._d2h = torch.cuda.Stream(), torch.cuda.Stream()
+        self._q = [torch.empty(q_host.shape[1:], dtype=q_host.dtype, device=dec.device)
+                   for _ in range(2)]
+        self._o = [torch.empty_like(dec.out) for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(steps)]
+        q_in = [torch.cuda.Event() for _ in range(steps)]
+        o_out = [torch.cuda.Event() for _ in range(steps)]
+        torch.cuda.synchronize()  # buffers made on other streams are ready
+        s, h2d, d2h = self.stream, self._h2d, self._d2h
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=s):
+            h2d.wait_stream(s)  # the copy streams join the capture
+            d2h.wait_stream(s)
+            for i in range(steps):
+                t = t0 + i
+                with torch.cuda.stream(h2d):
+                    if i >= 2:
+                        h2d.wait_event(done[i - 2])
+                    self._q[i % 2].copy_(q_host[t], non_blocking=True)
+                    q_in[i].record(h2d)
+                s.wait_event(q_in[i])
+                if i >= 2:
+                    s.wait_event(o_out[i - 2])
+                dec.step(t, self._q[i % 2], k, v, out=self._o[i % 2])
+                done[i].record(s)
+                with torch.cuda.stream(d2h):
+                    d2h.wait_event(done[i])
+                    out_host[i].copy_(self._o[i % 2], non_blocking=True)
+                    o_out[i].record(d2h)
+            s.wait_stream(h2d)
+            s.wait_stream(d2h)
+
+    def replay(self) -> None:
+        """Enqueues the loop on its stream (asynchronous: synchronise the
+        stream before reading out_host)."""
+        with torch.cuda.stream(self.stream):
+            self.graph.replay()

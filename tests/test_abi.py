@@ -187,3 +187,17 @@ def test_sequence_shard_call_validation(lib):
     # logits: workspace too small
     assert lib.saga_qk_logits(ctypes.byref(d), 16, 16, 16, base, need - 1, None) == \
         _lib.SAGA_ERR_WORKSPACE
+
+
+def test_host_loop_checks_its_buffers():
+    """The host loop refuses host buffers that do not cover its steps or are
+    not pinned, before it touches a device."""
+    from sparse_decode_attention_saga_b200.decoder import HostLoop
+    with pytest.raises(ValueError, match="cover"):
+        HostLoop(None, None, None, torch.zeros(4, 2), torch.zeros(2, 2), 0, 3)
+    with pytest.raises(ValueError, match="cover"):
+        HostLoop(None, None, None, torch.zeros(4, 2), torch.zeros(3, 2), 2, 3)
+    with pytest.raises(ValueError, match="cover"):
+        HostLoop(None, None, None, torch.zeros(4, 2), torch.zeros(3, 2), 0, 0)
+    with pytest.raises(ValueError, match="pinned"):
+        HostLoop(None, None, None, torch.zeros(4, 2), torch.zeros(3, 2), 0, 3)
