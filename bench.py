@@ -208,6 +208,31 @@ def oracle_sample_us_per_step(w, seed, steps_sample, t0):
     return us, oracle.num_threads(), desc
 
 
+def oracle_single_thread_us(w, seed, t0):
+    """The oracle's step t0 on one batch element on one host thread, scaled
+    to the whole batch (the state entering t0 is set up on all threads).
+    Returns (us_per_step, description)."""
+    import oracle  # test infrastructure: only this leg of the benchmark runs it
+    ws = w.scaled(batch=1)
+    K, V = make_cache(ws, seed)
+    qs = make_queries(ws, seed, steps=t0 + 1)
+    Kh, Vh = bf16_bits(K), bf16_bits(V)
+    tau = np.full((1, w.h_q), np.nan, np.float32)
+    t_last = (t0 // w.n) * w.n
+    if t_last < t0:
+        oracle.atopn_step(bf16_bits(qs[t_last]), Kh, Vh, tau, w.N, t_last, w.n)
+    threads = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        a = time.perf_counter()
+        oracle.atopn_step(bf16_bits(qs[t0]), Kh, Vh, tau, w.N, t0, w.n)
+        us = (time.perf_counter() - a) * 1e6 * w.batch
+    finally:
+        oracle.set_num_threads(threads)
+    return us, (f"oracle step {t0} on 1 of {w.batch} batch elements, one thread, "
+                f"scaled x{w.batch}")
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, world, rank):
@@ -565,8 +590,11 @@ def run_ours(args, world, rank, local):
     }
     if rank == 0 and not args.no_cpu_baseline:
         us_cpu, cores, desc = oracle_sample_us_per_step(w, args.seed, 2, w.n - 1)
+        us_one, desc_one = oracle_single_thread_us(w, args.seed, w.n - 1)
         line["cpu_baseline"] = {"value": us_cpu, "unit": "us/step", "cores": cores,
-                                "kind": "oracle", "sample": desc}
+                                "kind": "oracle", "sample": desc,
+                                "single_thread": {"value": us_one, "unit": "us/step",
+                                                  "sample": desc_one}}
     if not cold:
         del graph
     if rank == 0:
