@@ -11,7 +11,9 @@ runs steps 0..W-1; the timed region runs steps W..W+K-1 as one CUDA-graph
 replay ("compiled CUDA graphs", as in the pages' latency protocol), timed
 with CUDA events on the capture stream, max over ranks.  Inputs (K and V
 caches of 3 GB at the default workload) are larger than the 126 MB L2, so
-no flush is needed between steps.
+no flush is needed between steps; caches under 4x L2 are timed one graph per
+step with an L2 flush between.  The end-to-end leg runs the same steps
+through AtopNDecoder.host_loop (queries from, outputs to pinned host memory).
 
 Prints ONE JSON line (rank 0).  N > 1 runs independent replicas (one batch
 per GPU, no collective on the data path; weak scaling).
@@ -306,8 +308,8 @@ def run_ours(args, world, rank, local):
 
     # Caches that are not much larger than L2 are timed cold: every step is
     # its own CUDA graph, replayed between its own events with an L2 flush (a
-    # write larger than L2) outside them.  Larger caches stream past L2 anyway
-    # and are timed as one CUDA-graph replay of the K steps.
+    # write, then a read, each twice L2) outside them.  Larger caches stream
+    # past L2 anyway and are timed as one CUDA-graph replay of the K steps.
     cache_bytes = (K.numel() + V.numel()) * 2
     cold = cache_bytes < 4 * L2_BYTES
     flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if cold else None
