@@ -102,8 +102,10 @@ class HostLoop:
     two copy streams into and out of double buffers, so that they overlap the
     kernels of the neighbouring steps: query buffer t mod 2 is refilled once
     step t - 2 has run, and output buffer t mod 2 is rewritten once its copy
-    of step t - 2 is out.  The graph keeps the addresses of k, v and the host
-    buffers; replay() enqueues the whole loop on the loop's stream."""
+    of step t - 2 is out.  The graph keeps the addresses of k, v, the host
+    buffers and the decoder's state, so the loop holds references to all of
+    them; replay() enqueues the whole loop on the loop's stream (a side
+    stream: a capture cannot run on the default stream)."""
 
     def __init__(self, dec, k, v, q_host, out_host, t0, steps, stream=None):
         steps, t0 = int(steps), int(t0)
@@ -113,6 +115,7 @@ class HostLoop:
             raise ValueError("host buffers must be pinned")
         self.stream = torch.cuda.Stream() if stream is None else stream
         self.q_host, self.out_host = q_host, out_host
+        self._keep = (dec, k, v)  # the graph reads their memory on every replay
         self._h2d, self._d2h = torch.cuda.Stream(), torch.cuda.Stream()
         self._q = [torch.empty(q_host.shape[1:], dtype=q_host.dtype, device=dec.device)
                    for _ in range(2)]
