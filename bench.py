@@ -8,7 +8,7 @@ A step is one decode token of the Atop-N loop: refresh (exact radix select of
 the N-th largest logit) when t mod n == 0, otherwise the fused reuse step,
 always followed by the kept-entry softmax and gathered value sum.  Warm-up
 runs steps 0..W-1; the timed region runs steps W..W+K-1 as one CUDA-graph
-replay ("compiled CUDA graphs", as in the pages' latency protocol), timed
+replay (the pages time their decode loop as captured CUDA graphs), timed
 with CUDA events on the capture stream, max over ranks.  Inputs (K and V
 caches of 3 GB at the default workload) are larger than the 126 MB L2, so
 no flush is needed between steps; caches under 4x L2 are timed one graph per
@@ -346,6 +346,15 @@ def run_ours(args, world, rank, local):
     gpu_launches = _lib.launch_count() - before
     refresh_steps = sum(1 for t in range(args.warmup, total_steps) if t % w.n == 0)
 
+    # The untimed replays left the thresholds of the window's last refresh;
+    # put back those that enter step W (the refresh that opened its period),
+    # as in a decode that has just run steps 0..W-1.
+    t_open = args.warmup - args.warmup % w.n
+    if t_open < args.warmup:
+        with torch.cuda.stream(stream):
+            dec.refresh(qs[t_open], K)
+        stream.synchronize()
+
     sampler = ClockSampler(local)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -473,9 +482,14 @@ def run_ours(args, world, rank, local):
         # (AtopNDecoder.host_loop: each step's query copied in from pinned
         # host memory and its output copied out, on two copy streams with
         # double buffers, overlapping the neighbouring steps' kernels)
-        loop = dec.host_loop(K, V, q_host, out_host, args.warmup, args.steps, stream=stream)
+        # The thresholds entering step W (the refresh that opened its period)
+        # are put in place outside the timed region before each replay.
+        loop = dec.host_loop(K, V, q_host, out_host, args.warmup, args.steps, stream=stream,
+                             restore=False)
+        loop.restore_state()
         loop.replay()             # untimed: the first launch uploads the graph
         stream.synchronize()
+        loop.restore_state()
         with torch.cuda.stream(stream):
             e0.record(stream)
             loop.replay()
@@ -486,11 +500,13 @@ def run_ours(args, world, rank, local):
     else:
         # cold like the timed loop above: one host loop of one step per step,
         # L2 flushed before every step outside the events
-        loops = [dec.host_loop(K, V, q_host, out_host[k:k + 1], args.warmup + k, 1, stream=stream)
-                 for k in range(args.steps)]
+        loops = [dec.host_loop(K, V, q_host, out_host[k:k + 1], args.warmup + k, 1, stream=stream,
+                               restore=False) for k in range(args.steps)]
+        loops[0].restore_state()  # each later step follows its predecessor
         for lp in loops:          # untimed first launches, in step order
             lp.replay()
         stream.synchronize()
+        loops[0].restore_state()
         e2e_ms = 0.0
         for lp in loops:
             with torch.cuda.stream(stream):

@@ -67,6 +67,16 @@
 extern "C" {
 #endif
 
+/* Host-side state of the library (no device memory is allocated): per
+ * device, the device's properties and the kernels whose shared-memory limit
+ * has been raised on it (CUDA keeps that attribute per device); the launch
+ * counter (saga_launch_count); per host thread, the measurement events of
+ * saga_set_kernel_events; and, for saga_topn_refresh_noalloc, the device
+ * address of its scratch array per device.  All of it is filled on first use
+ * and guarded by mutexes.  It is not rebuilt after cudaDeviceReset: a process
+ * that resets a device must not call this library on that device again (its
+ * cached attributes and scratch address belong to the destroyed context). */
+
 /* Same type as cudaStream_t; 0 is the legacy default stream. */
 typedef struct CUstream_st* saga_stream_t;
 
@@ -97,16 +107,16 @@ typedef enum {
 size_t saga_workspace_bytes(const saga_dims* dims, int32_t N);
 
 /* Dense (full-attention) grouped-query decode: every cached position kept.
- * The speedup denominator ("baseline full attention", ai.info summary, Main
- * Findings, end-to-end speedups).  out[b,i,:] = softmax_j(s[b,i,j]) V[b,j,vh(i),:].
+ * The speedup denominator (ai.info summary, Main Findings: the end-to-end
+ * speedups are measured against full attention).  out[b,i,:] = softmax_j(s[b,i,j]) V[b,j,vh(i),:].
  * Split-K over l_kv (flash-decoding) followed by a log-sum-exp combine. */
 int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const void* v,
                       float* out, void* ws, size_t ws_bytes, saga_stream_t stream);
 
 /* Threshold refresh, run on steps with t mod n == 0 (the caller schedules).
  * thresh_out[b,i] = the exact N-th largest logit of row (b,i), counting
- * duplicates (Key Contributions #2: "exact top-N thresholds computed once
- * every n tokens"); N >= l_kv gives -inf (keep everything); a threshold of
+ * duplicates (Key Contributions #2: the exact threshold is found on every
+ * n-th token only); N >= l_kv gives -inf (keep everything); a threshold of
  * -0.0 is written as +0.0.
  *   logits_in  != NULL: use these logits [b,h_q,l_kv]; q and k are ignored.
  *   logits_in  == NULL: compute the logits from q and k; if logits_out is
@@ -118,7 +128,11 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
                       void* ws, size_t ws_bytes, saga_stream_t stream);
 
 /* One Atop-N decode step with the thresholds `thresh` (fresh from
- * saga_topn_refresh on refresh steps, reused otherwise):
+ * saga_topn_refresh on refresh steps, reused otherwise).  The kept set is
+ * found by a per-element comparison with the stored threshold, not by a sort
+ * (ai.info summary, Key Contributions #2; Methodology in Plain English ¶2),
+ * and only the kept value rows of value head vh(i) are read (Main Findings,
+ * "Bottleneck shift"; SAGA heads, Key Contributions #3):
  *   tau_eff = min(thresh[b,i], max_j s[b,i,j]);  keep j  <=>  s[b,i,j] >= tau_eff;
  *   out[b,i,:] = sum_kept softmax(s) V[b,j,vh(i),:].
  * The min() keeps the row's maximal entries when a stale threshold lies
@@ -132,12 +146,13 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
  *                      recomputes the same logits bit for bit with the same
  *                      tensor-core routine as saga_topn_refresh, so the kept
  *                      set is identical.
- *   logits_in == NULL and sel_idx == NULL: the fused kernel computes the
- *                      logits on chip, compares, and gathers only the kept
- *                      value rows; logits never reach device memory.
- *   logits_in == NULL and sel_idx != NULL: logits go through the workspace
- *                      so the kept positions can be emitted.
- * sel_idx (nullable): kept positions of each row, ascending.
+ *   logits_in == NULL: the fused kernel computes the logits on chip,
+ *                      compares, and gathers only the kept value rows;
+ *                      logits never reach device memory.  With sel_idx, one
+ *                      more kernel writes the positions that on-chip compare
+ *                      kept (the same kernels decide the output either way).
+ * sel_idx (nullable): kept positions of each row, ascending; entries past
+ *                     sel_cnt[b,i] are left as they were.
  * sel_cnt (nullable): number kept per row. */
 int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const void* v,
                       const float* thresh, const float* logits_in, float* out,

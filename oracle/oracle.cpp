@@ -150,7 +150,8 @@ int oracle_nth_largest_sort(const float* s, long rows, long l, long N, float* ta
 }
 
 // Step 3, selection by per-element comparison (Key Contributions #2 and
-// Methodology ¶2: a "cheap parallel comparison" instead of sorting).
+// Methodology ¶2: each logit is compared with the stored threshold; nothing
+// is sorted).
 //   tau_eff = min(tau, max_j s_j);  keep_j  <=>  s_j >= tau_eff.
 // mask: [rows,l] bytes (1 = kept); cnt: [rows] number kept.
 int oracle_select(const float* s, long rows, long l, const float* tau,
@@ -212,8 +213,9 @@ int oracle_attend_masked(long b, long hq, long hv, long d, long l, long l_cap,
     return bad ? -2 : 0;
 }
 
-// Full (dense) attention, the speedup denominator (Main Findings, "end-to-end
-// decoding speedups ... over baseline full attention"): every position kept.
+// Full (dense) attention, the speedup denominator (Main Findings: the
+// end-to-end speedups are measured against full attention): every position
+// kept.
 // dk: key/query head dim (logits), dv: value head dim (output).
 int oracle_decode_dense(long b, long hq, long hk, long hv, long dk, long dv, long l, long l_cap,
                         const uint16_t* q, const uint16_t* K, const uint16_t* V,

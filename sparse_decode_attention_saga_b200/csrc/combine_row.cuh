@@ -24,10 +24,12 @@ namespace saga {
 constexpr int kCombineThreads = 256;
 
 // raw: out_row gets the sum of the value rows at m_star instead of their
-// mean.  Returns their number (all lanes).
+// mean.  idx_out (nullable): their positions, ascending.  Returns their
+// number (all lanes).
 template <int DV, int D, int NT>  // D: key/query head dim, DV: value head dim
 __device__ int fallback_row(const CombineArgs& a, long long row, float m_star, float* out_row,
-                            int32_t* cnt_out, uint8_t* kbuf, bool raw = false) {
+                            int32_t* cnt_out, uint8_t* kbuf, bool raw = false,
+                            int32_t* idx_out = nullptr) {
     const Geometry& g = a.g;
     const int lane = threadIdx.x & 31;
     const int bb = static_cast<int>(row / g.hq);
@@ -78,6 +80,7 @@ __device__ int fallback_row(const CombineArgs& a, long long row, float m_star, f
                 const int src = __ffs(ball) - 1;
                 ball &= ball - 1;
                 const int pos = j0 + (src >> 2) + 8 * h;
+                if (idx_out && lane == 0) idx_out[count] = pos;  // ascending: h, then lane
                 const __nv_bfloat16* vr =
                     V + ((static_cast<size_t>(bb) * g.l_cap + pos) * g.hv + vh) * DV + lane * CPL;
 #pragma unroll
@@ -283,9 +286,10 @@ __device__ void merge_same_reference(const CombineArgs& a, long long row, int R,
     if (cnt == 0) {
         if (a.fallback) {
             if (warp == 0) {
-                const int c = fallback_row<D, DK, NT>(a, row, m_all, out_row,
-                                                      part || !a.sel_cnt ? nullptr : a.sel_cnt + row,
-                                                      kbuf, part != nullptr);
+                const int c = fallback_row<D, DK, NT>(
+                    a, row, m_all, out_row, part || !a.sel_cnt ? nullptr : a.sel_cnt + row, kbuf,
+                    part != nullptr,
+                    part || !a.sel_idx ? nullptr : a.sel_idx + static_cast<size_t>(row) * g.l);
                 if (part && lane == 0) {
                     part[0] = -kInf;
                     part[1] = static_cast<float>(c);

@@ -1,6 +1,6 @@
 // Dense grouped-query decode attention: the full-attention baseline the
 // speedups are measured against ("More Value per Key", ai.info summary, Main
-// Findings, end-to-end decoding speedups over baseline full attention).
+// Findings: the end-to-end speedups compare against full attention).
 //
 // Split-K (flash-decoding) over the flattened (batch, tile) space, same
 // partition as the streaming kernel.  The producer warp loads each tile's K
@@ -327,8 +327,7 @@ cudaError_t launch_t(const CUtensorMap& kmap, const CUtensorMap& vmap, const Den
                      cudaStream_t stream) {
     const size_t smem = dense_smem_bytes(a.g, a.stages);
     auto kern = dense_kernel<D, DV, NT, NCT>;
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem);
+    const cudaError_t attr = allow_dynamic_smem(kern, kMaxDynamicSmem);
     if (attr != cudaSuccess) return attr;
     if (smem > static_cast<size_t>(kMaxDynamicSmem)) return cudaErrorInvalidValue;
     kern<<<a.C, kStreamThreads, smem, stream>>>(kmap, vmap, a);

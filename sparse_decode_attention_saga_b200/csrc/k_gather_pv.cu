@@ -307,16 +307,6 @@ size_t gather_smem_bytes(int max_lists) {
     return (2 * static_cast<size_t>(max_lists) + 1) * sizeof(int);
 }
 
-// Lets both block orders of one instantiation use the list table's
-// dynamic shared memory (set once per instantiation).
-template <typename K>
-cudaError_t allow_table_smem(K k_rows, K k_parts) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(k_rows, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem);
-    return e != cudaSuccess
-               ? e
-               : cudaFuncSetAttribute(k_parts, cudaFuncAttributeMaxDynamicSharedMemorySize, kGatherMaxSmem);
-}
 
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
     const long long rows = static_cast<long long>(a.g.b) * a.g.hq;
@@ -330,10 +320,10 @@ cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
     if (a.g.dv == D_ && a.g.d == DK_ && a.g.NT == NT_) {                                       \
         auto k_rows = gather_pv_kernel<D_, DK_, NT_, false>;                                   \
         auto k_parts = gather_pv_kernel<D_, DK_, NT_, true>;                                   \
-        static const cudaError_t attr = allow_table_smem(k_rows, k_parts);                     \
+        auto kern = a.part_major ? k_parts : k_rows;                                           \
+        const cudaError_t attr = allow_dynamic_smem(kern, kGatherMaxSmem);                     \
         if (attr != cudaSuccess) return attr;                                                  \
-        return launch_dependent(a.part_major ? k_parts : k_rows, grid, dim3(kThreads), smem,   \
-                                stream, a);                                                    \
+        return launch_dependent(kern, grid, dim3(kThreads), smem, stream, a);                  \
     }
     SAGA_GATHER_CASE(64, 64, 1)
     SAGA_GATHER_CASE(64, 64, 2)

@@ -316,9 +316,7 @@ template <int D, int NT, int MODE>
 cudaError_t launch_t(const CUtensorMap& kmap, const StreamArgs& a, cudaStream_t stream) {
     const size_t smem = stream_smem_bytes(a.stages);
     auto kern = qk_stream_kernel<D, NT, MODE>;
-    // once per instantiation, so launches inside a stream capture set nothing
-    static const cudaError_t attr = cudaFuncSetAttribute(
-        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynamicSmem);
+    const cudaError_t attr = allow_dynamic_smem(kern, kMaxDynamicSmem);
     if (attr != cudaSuccess) return attr;
     kern<<<a.C, kStreamThreads, smem, stream>>>(kmap, a);
     return cudaGetLastError();

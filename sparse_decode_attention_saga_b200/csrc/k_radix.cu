@@ -2,7 +2,8 @@
 // head) row, counting duplicates.
 //
 // Method: "More Value per Key" (ai.info summary, Key Contributions #2): Atop-N
-// reuses exact top-N thresholds computed once every n tokens.  The pages do
+// finds the exact N-th largest logit only on every n-th token and reuses
+// that threshold on the tokens in between.  The pages do
 // not say how the exact threshold is found; this is an MSB-first radix select
 // on order-preserving 32-bit keys (digits of 11, 11 and 10 bits), which is
 // exact and needs no sort.

@@ -142,7 +142,87 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
     if (tid == 0) a.cnt[row] = total;
 }
 
+// One CTA per row: clear the row's bitmap, set the bit of every listed
+// position (a position is listed at most once per row), then each thread
+// takes a contiguous run of bitmap words and writes their set positions at
+// its offset from a block scan of the runs' counts, which yields the row's
+// kept positions in ascending order.
+__global__ void __launch_bounds__(kThreads) lists_to_index_kernel(const IndexArgs a) {
+    __shared__ int warp_tot[kWarps];
+    pdl_wait();  // the lists come from the fused kernel, two launches back
+    const Geometry& g = a.g;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long row = blockIdx.x;
+    const int bb = static_cast<int>(row / g.hq);
+    const long long T = static_cast<long long>(g.b) * g.tiles;
+    const int nl = slots_of_batch(bb, g.tiles, T, a.C) * g.WPK;
+    const int32_t* cnt = a.seg_cnt + static_cast<size_t>(row) * g.S_cap * g.WPK;
+    auto clamped = [&](int j, SegList& sl) {
+        sl = seg_list_of(g.P, g.MBW, g.WPK, g.tiles, bb, j, T, a.C);
+        return min(max(__ldg(cnt + j), 0), sl.cap);
+    };
+    int mine = 0;
+    for (int j = tid; j < nl; j += kThreads) {
+        SegList sl;
+        mine += clamped(j, sl);
+    }
+    mine = __reduce_add_sync(0xffffffffu, mine);
+    if (lane == 0) warp_tot[warp] = mine;
+    __syncthreads();
+    int total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) total += warp_tot[w];
+    if (total == 0) return;  // the empty-set fallback of the row merge writes this row
+
+    const int words = (g.l + 31) >> 5;
+    uint32_t* bm = a.bitmap + static_cast<size_t>(row) * words;
+    for (int w = tid; w < words; w += kThreads) bm[w] = 0u;
+    __syncthreads();
+    const int2* lists = a.seg_list + static_cast<size_t>(row) * g.l_pad;
+    for (int j = warp; j < nl; j += kWarps) {
+        SegList sl;
+        const int n = clamped(j, sl);
+        for (int e = lane; e < n; e += 32) {
+            const int pos = __ldg(&lists[sl.start + e].x);
+            if (pos >= 0 && pos < g.l) atomicOr(bm + (pos >> 5), 1u << (pos & 31));
+        }
+    }
+    __syncthreads();
+
+    const int per = (words + kThreads - 1) / kThreads;
+    const int w0 = min(words, tid * per), w1 = min(words, w0 + per);
+    int c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(__ldcg(bm + w));
+    int inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
+    }
+    __syncthreads();
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    int at = inc - c;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) at += w < warp ? warp_tot[w] : 0;
+    int32_t* dst = a.idx + static_cast<size_t>(row) * g.l;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t bits = __ldcg(bm + w);
+        while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            dst[at++] = (w << 5) + b;
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_lists_to_index(const IndexArgs& a, cudaStream_t stream) {
+    const long long rows = static_cast<long long>(a.g.b) * a.g.hq;
+    return launch_dependent(lists_to_index_kernel, dim3(static_cast<unsigned>(rows)), dim3(kThreads), 0,
+                            stream, a);
+}
 
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream) {
     const bool vec = (a.l % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.logits) & 15u) == 0);

@@ -279,6 +279,40 @@ int run_logits(const Geometry& g, const DeviceInfo& dev, const void* q, const vo
 
 namespace saga {
 void note_launches(int n) { g_launches += static_cast<uint64_t>(n); }
+
+namespace {
+// (kernel, limit) pairs whose attribute has been set, with a bit per device.
+struct SmemAttr {
+    const void* fn;
+    int bytes;
+    uint64_t devices;
+};
+constexpr int kMaxSmemAttrs = 128;
+SmemAttr g_smem_attr[kMaxSmemAttrs];
+int g_n_smem_attr = 0;
+std::mutex g_smem_attr_mu;
+}  // namespace
+
+cudaError_t allow_dynamic_smem(const void* fn, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const uint64_t bit = 1ull << dev;
+    std::lock_guard<std::mutex> lock(g_smem_attr_mu);
+    SmemAttr* rec = nullptr;
+    for (int i = 0; i < g_n_smem_attr; ++i)
+        if (g_smem_attr[i].fn == fn && g_smem_attr[i].bytes == bytes) rec = &g_smem_attr[i];
+    if (rec && (rec->devices & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    if (!rec && g_n_smem_attr < kMaxSmemAttrs) {
+        rec = &g_smem_attr[g_n_smem_attr++];
+        *rec = SmemAttr{fn, bytes, 0};
+    }
+    if (rec) rec->devices |= bit;  // (a full table only means setting it again next time)
+    return cudaSuccess;
+}
 }  // namespace saga
 
 extern "C" {
@@ -376,14 +410,9 @@ static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k
         aligned(q, 16) && aligned(k, 16))
         logits_in = nullptr;
 
-    if (logits_in || sel_idx) {
+    if (logits_in) {
         // stored logits -> compare/compact -> gathered PV -> combine
         const float* logits = logits_in;
-        if (!logits) {
-            float* dst = ws_at<float>(ws, L.logits);
-            if ((st = run_logits(g, dev, q, k, dst, err, s))) return st;
-            logits = dst;
-        }
         SelectArgs sa{};
         sa.logits = logits;
         sa.thresh = thresh;
@@ -479,8 +508,21 @@ static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k
     ga.cmb.out = out;
     ga.cmb.part = part;
     ga.cmb.sel_cnt = sel_cnt;
+    ga.cmb.sel_idx = sel_idx;
     g_launches += 1;
-    return cuda_status(launch_gather_pv(ga, s));
+    if ((e = launch_gather_pv(ga, s)) != cudaSuccess || !sel_idx) return cuda_status(e);
+
+    // the kept positions of the on-chip compare, ascending (the logits region
+    // of the workspace, unused on this path, holds the per-row bitmaps)
+    IndexArgs ia{};
+    ia.g = g;
+    ia.C = a.C;
+    ia.seg_list = a.list;
+    ia.seg_cnt = a.seg_cnt;
+    ia.bitmap = ws_at<uint32_t>(ws, L.logits);
+    ia.idx = sel_idx;
+    g_launches += 1;
+    return cuda_status(launch_lists_to_index(ia, s));
 }
 
 int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const void* v,

@@ -30,6 +30,16 @@ cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// Raises the dynamic shared-memory limit of kernel `fn` to `bytes` on the
+// current device.  CUDA keeps function attributes per device, so this is
+// done once per (kernel, device) and remembered (a process that drives
+// several GPUs sets it on each before the kernel's first launch there).
+cudaError_t allow_dynamic_smem(const void* fn, int bytes);
+template <typename... KArgs>
+cudaError_t allow_dynamic_smem(void (*kern)(KArgs...), int bytes) {
+    return allow_dynamic_smem(reinterpret_cast<const void*>(kern), bytes);
+}
+
 // Streaming query-key kernel over the K cache (TMA pipeline + mma).
 enum StreamMode : int {
     kStreamLogits = 0,  // write s = q.k/sqrt(d) to logits [b,hq,l]
@@ -94,6 +104,20 @@ struct SelectArgs {
 };
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream);
 
+// Ascending kept positions of every row from the fused kernel's per-(slot,
+// warp) lists: the lists' positions are set in a per-row bitmap, which is
+// then compacted in position order.  Rows that kept nothing are skipped (the
+// row merge's empty-set fallback writes their positions).
+struct IndexArgs {
+    Geometry g;
+    int C;                   // grid of the fused kernel
+    const int2* seg_list;    // (position, logit bits) pairs [rows][l_pad]
+    const int32_t* seg_cnt;  // [rows][S_cap][WPK]
+    uint32_t* bitmap;        // scratch [rows][ceil(l/32)]
+    int32_t* idx;            // [rows][l] out
+};
+cudaError_t launch_lists_to_index(const IndexArgs& a, cudaStream_t stream);
+
 // Log-sum-exp merge of partial records, plus the empty-set fallback.
 enum CombineMode : int {
     kCombineParts = 0,     // `parts` records per row (gathered contiguous lists)
@@ -115,6 +139,9 @@ struct CombineArgs {
     const float* records;
     float* out;
     int32_t* sel_cnt;
+    // Optional: [rows][l] kept positions; written here only for rows that
+    // kept nothing (the empty-set fallback's positions at the row maximum)
+    int32_t* sel_idx;
     // Optional, for a sequence shard: the row's merged but unnormalised
     // record (m, l, count, row max, o[dv]) goes to part[row] instead of out
     // (count 0: m = -inf, l = number of positions at the row max, o = the

@@ -66,6 +66,23 @@ SAGA_HD int slots_of_batch(int bb, int tiles, long long T, int C) {
     return cta_of_tile(x0 + tiles - 1, T, C) - cta_of_tile(x0, T, C) + 1;
 }
 
+// List j (= slot * WPK + warp) of batch row bb in the fused kernel's kept
+// lists: the offset of its first entry in the row's list region and the
+// number of entries it can hold (the warp's share of the slot's positions).
+struct SegList {
+    int start, cap;
+};
+SAGA_HD SegList seg_list_of(int P, int MBW, int WPK, int tiles, int bb, int j, long long T, int C) {
+    const long long x0 = static_cast<long long>(bb) * tiles;
+    const int sl = j / WPK, sub = j - sl * WPK;
+    const int c = cta_of_tile(x0, T, C) + sl;
+    const long long t0 = cta_tile_begin(T, C, c), t1 = cta_tile_begin(T, C, c + 1);
+    const long long s0 = t0 > x0 ? t0 : x0;
+    const long long s1 = t1 < x0 + tiles ? t1 : x0 + tiles;
+    const int cap = static_cast<int>((s1 - s0) * MBW * 16);
+    return SegList{static_cast<int>((s0 - x0) * P) + sub * cap, cap};
+}
+
 // The regions up to `rowmax` depend only on the batch and head counts, so
 // their offsets do not move when the cached length changes (decode with a
 // growing cache); the per-row tickets, which must be zero on entry, live

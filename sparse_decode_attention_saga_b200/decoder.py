@@ -3,7 +3,8 @@
 ``AtopNDecoder`` owns the caller-side state the method needs (the threshold
 tensor, the workspace and a logits buffer for refresh steps) and applies the
 refresh schedule of "More Value per Key" (ai.info summary, Key Contributions
-#2: exact top-N thresholds computed once every n tokens and reused between):
+#2: the exact threshold is recomputed on every n-th token only and reused on
+the tokens in between):
 step t refreshes when t mod n == 0, then decodes with the stored thresholds.
 Every step is two or three C calls; all compute runs in libsaga.so.
 ``HostLoop`` (``AtopNDecoder.host_loop``) runs a span of steps as one CUDA
@@ -88,11 +89,12 @@ class AtopNDecoder:
     def error(self, stream=None) -> int:
         return _lib.workspace_error(self.ws, stream)
 
-    def host_loop(self, k, v, q_host, out_host, t0: int, steps: int, stream=None) -> "HostLoop":
+    def host_loop(self, k, v, q_host, out_host, t0: int, steps: int, stream=None,
+                  restore: bool = True) -> "HostLoop":
         """Captures decode steps t0 .. t0 + steps - 1 fed from pinned host
         memory (see HostLoop); the decoder must have run a step outside a
         capture first, and its cached length stays fixed inside the loop."""
-        return HostLoop(self, k, v, q_host, out_host, t0, steps, stream)
+        return HostLoop(self, k, v, q_host, out_host, t0, steps, stream, restore)
 
 
 class HostLoop:
@@ -105,9 +107,18 @@ class HostLoop:
     of step t - 2 is out.  The graph keeps the addresses of k, v, the host
     buffers and the decoder's state, so the loop holds references to all of
     them; replay() enqueues the whole loop on the loop's stream (a side
-    stream: a capture cannot run on the default stream)."""
+    stream: a capture cannot run on the default stream).
 
-    def __init__(self, dec, k, v, q_host, out_host, t0, steps, stream=None):
+    Thresholds entering t0: the steps before the loop's first refresh reuse
+    the thresholds of the refresh that opened t0's period (step t0 - t0 mod n,
+    from q_host of that step).  With restore=True (default) and t0 not a
+    refresh step, that refresh heads the graph, so every replay gives the
+    outputs of running steps t0 - t0 mod n .. t0 + steps - 1 one by one.
+    With restore=False the graph holds only the loop's own steps and the
+    caller puts that state in place before each replay (restore_state(), or
+    the steps before t0 run on the same decoder)."""
+
+    def __init__(self, dec, k, v, q_host, out_host, t0, steps, stream=None, restore=True):
         steps, t0 = int(steps), int(t0)
         if steps < 1 or t0 < 0 or q_host.shape[0] < t0 + steps or out_host.shape[0] < steps:
             raise ValueError("host buffers do not cover the steps")
@@ -115,10 +126,12 @@ class HostLoop:
             raise ValueError("host buffers must be pinned")
         self.stream = torch.cuda.Stream() if stream is None else stream
         self.q_host, self.out_host = q_host, out_host
+        self.t0, self.t_open = t0, t0 - t0 % dec.n  # step whose refresh holds for t0
         self._keep = (dec, k, v)  # the graph reads their memory on every replay
         self._h2d, self._d2h = torch.cuda.Stream(), torch.cuda.Stream()
         self._q = [torch.empty(q_host.shape[1:], dtype=q_host.dtype, device=dec.device)
                    for _ in range(2)]
+        self._q_open = torch.empty(q_host.shape[1:], dtype=q_host.dtype, device=dec.device)
         self._o = [torch.empty_like(dec.out) for _ in range(2)]
         done = [torch.cuda.Event() for _ in range(steps)]
         q_in = [torch.cuda.Event() for _ in range(steps)]
@@ -127,6 +140,8 @@ class HostLoop:
         s, h2d, d2h = self.stream, self._h2d, self._d2h
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph, stream=s):
+            if restore and self.t_open < t0:
+                self._open_period(s)
             h2d.wait_stream(s)  # the copy streams join the capture
             d2h.wait_stream(s)
             for i in range(steps):
@@ -147,6 +162,20 @@ class HostLoop:
                     o_out[i].record(d2h)
             s.wait_stream(h2d)
             s.wait_stream(d2h)
+
+    def _open_period(self, s) -> None:
+        """The refresh of step t_open on stream s (its query from q_host)."""
+        dec, k, _ = self._keep
+        with torch.cuda.stream(s):
+            self._q_open.copy_(self.q_host[self.t_open], non_blocking=True)
+            dec.refresh(self._q_open, k)
+
+    def restore_state(self) -> None:
+        """Enqueues, outside the graph, the refresh that opened t0's period
+        (nothing when t0 is a refresh step): the state a loop built with
+        restore=False expects at the start of each replay."""
+        if self.t_open < self.t0:
+            self._open_period(self.stream)
 
     def replay(self) -> None:
         """Enqueues the loop on its stream (asynchronous: synchronise the

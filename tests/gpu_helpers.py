@@ -83,3 +83,28 @@ def gpu_step_with_mask(dec: AtopNDecoder, t, q, K, V):
 
 def bits(t: torch.Tensor) -> np.ndarray:
     return bf16_bits(t)
+
+
+def gpu_logits(dec: AtopNDecoder, q, K) -> torch.Tensor:
+    """This step's logits [b, h_q, l_kv] from the library's logits kernel,
+    which shares its tensor-core routine with the fused compare."""
+    d = dec.dims
+    s = torch.empty((d.batch, d.h_q, d.l_kv), dtype=torch.float32, device="cuda")
+    _lib.qk_logits(d, q, K, s, dec.ws)
+    return s
+
+
+def assert_mask_exact(dec: AtopNDecoder, q, K, idx, cnt, rows=None, what=""):
+    """The kept positions a decode step emitted equal, bit for bit, the
+    oracle's selection over the GPU's own logits of that step and the
+    thresholds it used (identical logits must give identical masks)."""
+    s = gpu_logits(dec, q, K)
+    torch.cuda.synchronize()
+    sel = list(range(s.shape[0])) if rows is None else list(rows)
+    s_h = s[sel].cpu().numpy()
+    tau = dec.thresh[sel].cpu().numpy()
+    mask_ref, cnt_ref = oracle.select(s_h, tau)
+    got_cnt = cnt[sel].cpu().numpy()
+    assert np.array_equal(got_cnt, cnt_ref), f"{what}: kept counts differ in {(got_cnt != cnt_ref).sum()} rows"
+    mask_gpu = mask_from_lists(idx[sel], cnt[sel], s_h.shape[-1])
+    assert np.array_equal(mask_gpu, mask_ref), f"{what}: {(mask_gpu != mask_ref).sum()} mask entries differ"

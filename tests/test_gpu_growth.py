@@ -13,7 +13,7 @@ from sparse_decode_attention_saga_b200.decoder import AtopNDecoder
 from sparse_decode_attention_saga_b200.workload import Workload, make_new_rows
 
 from .gpu_helpers import (assert_mask_within_band, assert_outputs_close, bits, device_inputs,
-                          gpu_step_with_mask, mask_from_lists)
+                          gpu_step_with_mask, mask_from_lists, assert_mask_exact)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +48,7 @@ def _growth_loop(w: Workload, seed: int):
                                                        l=l)
         mask_gpu = mask_from_lists(idx, cnt, l)
         assert np.array_equal(cnt_f.cpu().numpy(), cnt.cpu().numpy()), f"t={t}"
+        assert_mask_exact(dec, qs[t], K, idx, cnt, what=f"t={t}")
         assert_mask_within_band(mask_gpu, m_ref, s_ref, tau_ref, f"t={t}")
         ref = oracle.attend_masked(s_ref, mask_gpu, Vh)
         assert_outputs_close(out_l.cpu().numpy(), ref, f"t={t} stored-logits")

@@ -2,7 +2,7 @@
 their outputs written to pinned host memory (one CUDA graph; the copies on
 two copy streams with double buffers) give, bit for bit, the outputs of the
 same steps run one by one on device buffers, and the same again on a second
-replay."""
+replay, also when the loop starts inside a refresh period."""
 import pytest
 import torch
 
@@ -18,9 +18,11 @@ if not torch.cuda.is_available():  # collected on CPU machines, selected out by -m 
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 
-@pytest.mark.parametrize("t0,steps", [(0, 1), (0, 2), (3, 7), (6, 12)],
-                         ids=["one", "two", "from_3_seven", "from_6_twelve"])
-def test_host_loop_matches_device_steps(t0, steps):
+@pytest.mark.parametrize("restore", [True, False], ids=["restore_in_graph", "restore_state"])
+@pytest.mark.parametrize("t0,steps", [(0, 1), (0, 2), (3, 7), (6, 12), (4, 5), (2, 1)],
+                         ids=["one", "two", "from_3_seven", "from_6_twelve", "mid_period_4_five",
+                              "mid_period_2_one"])
+def test_host_loop_matches_device_steps(t0, steps, restore):
     w = Workload("host_loop", 2, 8, 2, 4, 64, 1000, 25, 3, steps=t0 + steps)
     qs, K, V = device_inputs(w, seed=61)
     ref = AtopNDecoder.for_workload(w)
@@ -30,13 +32,17 @@ def test_host_loop_matches_device_steps(t0, steps):
         if t >= t0:
             expect.append(o.cpu())
     dec = AtopNDecoder.for_workload(w)
-    dec.step(0, qs[0], K, V)  # one call outside a capture; t0 is a refresh step
+    dec.step(0, qs[0], K, V)  # one call outside a capture
+    # thresholds that belong to no step of this loop: a replay must not use them
+    dec.thresh.fill_(0.5)
     q_host = qs.cpu().pin_memory()
     out_host = torch.empty((steps,) + tuple(dec.out.shape), dtype=torch.float32).pin_memory()
     torch.cuda.synchronize()
-    loop = dec.host_loop(K, V, q_host, out_host, t0, steps)
+    loop = dec.host_loop(K, V, q_host, out_host, t0, steps, restore=restore)
     for rep in range(2):
         out_host.fill_(float("nan"))
+        if not restore:
+            loop.restore_state()
         loop.replay()
         loop.stream.synchronize()
         for i in range(steps):

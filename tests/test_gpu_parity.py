@@ -14,8 +14,9 @@ from sparse_decode_attention_saga_b200 import _lib
 from sparse_decode_attention_saga_b200.decoder import AtopNDecoder
 from sparse_decode_attention_saga_b200.workload import CONFIGS, Workload
 
-from .gpu_helpers import (LOGIT_ATOL, LOGIT_RTOL, assert_mask_within_band, assert_outputs_close,
-                          bits, device_inputs, gpu_step_with_mask, mask_from_lists)
+from .gpu_helpers import (LOGIT_ATOL, LOGIT_RTOL, assert_mask_exact, assert_mask_within_band,
+                          assert_outputs_close, bits, device_inputs, gpu_logits, gpu_step_with_mask,
+                          mask_from_lists)
 
 pytestmark = pytest.mark.gpu
 
@@ -114,6 +115,44 @@ def test_mask_bit_exact_and_output_given_mask(shape):
     assert_outputs_close(out.cpu().numpy(), ref, "refresh-step output")
 
 
+@pytest.mark.parametrize("pick", ["rank_N", "random"])
+def test_fused_mask_exact_at_threshold_boundaries(shape, pick):
+    """Thresholds equal to one of the row's logits, or one ulp above or below
+    it: the fused kernel compares the raw tensor-core accumulator with a
+    threshold mapped back through the 1/sqrt(d) scale, and must keep exactly
+    what comparing the scaled logits keeps (head dim 128: the scale is not a
+    power of two)."""
+    w = shape
+    qs, K, V = device_inputs(w, seed=13, steps=1)
+    dec = AtopNDecoder.for_workload(w)
+    s = gpu_logits(dec, qs[0], K)
+    torch.cuda.synchronize()
+    sh = s.cpu().numpy()
+    if pick == "rank_N":
+        j = np.minimum(w.N, w.l_kv) - 1
+        base = -np.sort(-sh, axis=-1)[..., j]
+    else:
+        rng = np.random.default_rng(w.l_kv)
+        j = rng.integers(0, w.l_kv, size=(w.batch, w.h_q))
+        base = np.take_along_axis(sh, j[..., None], -1)[..., 0]
+    s_ref = oracle.logits(bits(qs[0]), bits(K), l=w.l_kv)
+    for kind, tau in (("at", base), ("above", np.nextafter(base, np.float32(np.inf))),
+                      ("below", np.nextafter(base, np.float32(-np.inf)))):
+        tau = tau.astype(np.float32)
+        dec.thresh.copy_(torch.from_numpy(tau))
+        out = torch.empty_like(dec.out)
+        idx = torch.full((w.batch, w.h_q, w.l_kv), -1, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros((w.batch, w.h_q), dtype=torch.int32, device="cuda")
+        _lib.atopn_decode(dec.dims, qs[0], K, V, dec.thresh, None, out, idx, cnt, dec.ws)
+        torch.cuda.synchronize()
+        mask_ref, cnt_ref = oracle.select(sh, tau)
+        assert np.array_equal(cnt.cpu().numpy(), cnt_ref), kind
+        mask_gpu = mask_from_lists(idx, cnt, w.l_kv)
+        assert np.array_equal(mask_gpu, mask_ref), f"{kind}: {(mask_gpu != mask_ref).sum()} differ"
+        assert_outputs_close(out.cpu().numpy(), oracle.attend_masked(s_ref, mask_gpu, bits(V)), kind)
+    assert dec.error() == _lib.SAGA_OK
+
+
 def test_stale_threshold_above_every_logit_keeps_the_maxima(shape):
     w = shape
     qs, K, V = device_inputs(w, seed=5, steps=2)
@@ -125,7 +164,9 @@ def test_stale_threshold_above_every_logit_keeps_the_maxima(shape):
     # fused path (fallback in the combine kernel)
     out_fused = torch.empty_like(dec.out)
     cnt_fused = torch.zeros((w.batch, w.h_q), dtype=torch.int32, device="cuda")
-    _lib.atopn_decode(dec.dims, qs[0], K, V, dec.thresh, None, out_fused, None, cnt_fused, dec.ws)
+    idx_fused = torch.full((w.batch, w.h_q, w.l_kv), -1, dtype=torch.int32, device="cuda")
+    _lib.atopn_decode(dec.dims, qs[0], K, V, dec.thresh, None, out_fused, idx_fused, cnt_fused,
+                      dec.ws)
     # stored-logits path
     out_l, idx, cnt = torch.empty_like(dec.out), None, None
     idx = torch.full((w.batch, w.h_q, w.l_kv), -1, dtype=torch.int32, device="cuda")
@@ -135,6 +176,7 @@ def test_stale_threshold_above_every_logit_keeps_the_maxima(shape):
     mask_ref, cnt_ref = oracle.select(s, dec.thresh.cpu().numpy())
     assert np.array_equal(mask_from_lists(idx, cnt, w.l_kv), mask_ref)
     assert np.array_equal(cnt_fused.cpu().numpy(), cnt_ref)
+    assert np.array_equal(mask_from_lists(idx_fused, cnt_fused, w.l_kv), mask_ref)
     ref = oracle.attend_masked(s, mask_ref, bits(V))
     assert_outputs_close(out_l.cpu().numpy(), ref, "stored-logits fallback")
     assert_outputs_close(out_fused.cpu().numpy(), ref, "fused fallback")
@@ -144,8 +186,13 @@ def test_stale_threshold_above_every_logit_keeps_the_maxima(shape):
 # ---------------------------------------------------------------- whole loop
 
 def run_loop_and_compare(w, seed=0, gen_device="cuda", rows=None):
-    """Steps 0..steps-1 on the GPU (fused reuse path + stored-logits path for
-    the mask) and in the oracle; returns number of in-band mask flips."""
+    """Steps 0..steps-1 on the GPU and in the oracle; returns the number of
+    in-band mask flips.  Each step runs twice: without and with the kept
+    positions emitted.  On reuse steps both runs take the fused path (the
+    on-chip compare of the streaming kernel), on refresh steps the
+    stored-logits path; either way the emitted mask is checked bit for bit
+    against the oracle's selection over the GPU's own logits, and against
+    the oracle's end-to-end step within the band."""
     qs, K, V = device_inputs(w, seed, gen_device=gen_device)
     dec = AtopNDecoder.for_workload(w)
     b_sel = list(range(w.batch)) if rows is None else rows
@@ -163,8 +210,11 @@ def run_loop_and_compare(w, seed=0, gen_device="cuda", rows=None):
         o_ref, s_ref, m_ref, c_ref = oracle.atopn_step(bits(qs[t][b_sel]), Kh, Vh, tau_ref,
                                                        w.N, t, w.n, l=w.l_kv)
         mask_gpu = mask_from_lists(idx[b_sel], cnt[b_sel], w.l_kv)
-        # the fused kernel keeps exactly what the stored-logits path keeps
+        # the same kernels decide the output whether or not the positions are emitted
         assert np.array_equal(cnt_fused[b_sel].cpu().numpy(), cnt[b_sel].cpu().numpy()), f"t={t}"
+        if not dec.is_refresh(t):
+            assert torch.equal(out_fused, out_l), f"t={t}: emitting positions changed the output"
+        assert_mask_exact(dec, qs[t], K, idx, cnt, b_sel, f"t={t}")
         flips += assert_mask_within_band(mask_gpu, m_ref, s_ref, tau_ref, f"t={t}")
         ref = oracle.attend_masked(s_ref, mask_gpu, Vh)
         assert_outputs_close(out_l[b_sel].cpu().numpy(), ref, f"t={t} stored-logits")
@@ -236,16 +286,24 @@ def test_zero_query_and_unit_values():
     np.testing.assert_allclose(out_f.cpu().numpy(), 1.0, rtol=1e-6)
 
 
-def test_same_query_reuse_is_bit_identical_to_refresh():
+def test_same_query_reuse_keeps_the_refresh_mask():
+    """A reuse step with the refresh step's own query keeps exactly the
+    refresh step's set: the fused on-chip compare (reuse) against the
+    stored-logits compare (refresh).  The outputs sum the same entries in a
+    different order, so they agree to rounding."""
     w = wl("same", 2, 32, 4, 8, 64, 5000, None, N=100, n=4, steps=1)
     qs, K, V = device_inputs(w, seed=11, steps=1)
     dec = AtopNDecoder.for_workload(w)
     o_ref, i_ref, c_ref = gpu_step_with_mask(dec, 0, qs[0], K, V)
     o_reu, i_reu, c_reu = gpu_step_with_mask(dec, 1, qs[0], K, V)
+    o_again, i_again, c_again = gpu_step_with_mask(dec, 2, qs[0], K, V)
     torch.cuda.synchronize()
     assert torch.equal(c_ref, c_reu)
     assert torch.equal(i_ref, i_reu)
-    assert torch.equal(o_ref, o_reu)
+    torch.testing.assert_close(o_reu, o_ref, rtol=1e-5, atol=1e-6)
+    # the fused path is deterministic
+    assert torch.equal(i_reu, i_again) and torch.equal(c_reu, c_again)
+    assert torch.equal(o_reu, o_again)
 
 
 def test_resume_from_saved_state_is_bit_identical():
