@@ -156,7 +156,8 @@ __device__ void combine_row(const CombineArgs& a, long long row, int r_begin = 0
     float* out_row = a.out + static_cast<size_t>(row) * D;
     if (cnt == 0 && a.fallback && !partial_out) {
         if (warp == 0)
-            fallback_row<D, DK, NT>(a, row, mall, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf);
+            fallback_row<D, DK, NT>(a, row, mall, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf,
+                                    false, a.sel_idx ? a.sel_idx + static_cast<size_t>(row) * g.l : nullptr);
         return;
     }
 

@@ -23,25 +23,13 @@
 #include "qk_tile.cuh"
 #include "saga_kernels.h"
 
+#ifndef SAGA_STREAM_K_HINT
+#define SAGA_STREAM_K_HINT 1
+#endif
+
 namespace saga {
 
 namespace {
-
-// Smallest fp32 x with fl(x * scale) >= tau.  fl(x * scale) is monotone in x,
-// so "x >= raw_threshold(tau, scale)" decides exactly what "fl(x * scale) >=
-// tau" decides, with one compare on the raw tensor-core accumulator.  The
-// start fl(tau / scale) is within two ulps of the boundary.
-__device__ __forceinline__ float raw_threshold(float tau, float scale) {
-    float x = __fdiv_rn(tau, scale);
-    if (!(x == x)) return x;  // NaN threshold: nothing compares >= it
-    for (int i = 0; i < 4 && __fmul_rn(x, scale) >= tau; ++i) {
-        const float below = nextafterf(x, -kInf);
-        if (__fmul_rn(below, scale) < tau) break;
-        x = below;
-    }
-    for (int i = 0; i < 4 && __fmul_rn(x, scale) < tau; ++i) x = nextafterf(x, kInf);
-    return x;
-}
 
 template <int D, int NT, int MODE>
 __global__ void __launch_bounds__(kStreamThreads, 2)
@@ -81,6 +69,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
             // K is read once per step: its lines go first, so that the kept
             // lists and logits written meanwhile stay in L2 for the next kernel
             const uint64_t k_policy = l2_policy_evict_first();
+            (void)k_policy;
             int issued = 0;
             int bb = static_cast<int>(t0 / g.tiles);
             int tl = static_cast<int>(t0 - static_cast<long long>(bb) * g.tiles);
@@ -93,8 +82,13 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
                 uint8_t* dst = smem + static_cast<size_t>(st) * kStageBytes;
                 for (int kh = 0; kh < g.hk; ++kh)
                     for (int dh = 0; dh < KTile<D>::NBOX; ++dh)
+#if SAGA_STREAM_K_HINT
                         tma_load_3d_hint(dst + (kh * KTile<D>::NBOX + dh) * g.P * KTile<D>::ROWB,
                                          &kmap, &full[st], dh * 64, kh, z, k_policy);
+#else
+                        tma_load_3d(dst + (kh * KTile<D>::NBOX + dh) * g.P * KTile<D>::ROWB,
+                                    &kmap, &full[st], dh * 64, kh, z);
+#endif
                 issued = k + 1;
                 if (++tl == g.tiles) {
                     tl = 0;

@@ -95,4 +95,20 @@ __device__ __forceinline__ void qk_mma(uint32_t tile, int rows_per_box, int kh, 
     }
 }
 
+// Smallest fp32 x with fl(x * scale) >= tau.  fl(x * scale) is monotone in x,
+// so "x >= raw_threshold(tau, scale)" decides exactly what "fl(x * scale) >=
+// tau" decides, with one compare on the raw tensor-core accumulator.  The
+// start fl(tau / scale) is within two ulps of the boundary.
+__device__ __forceinline__ float raw_threshold(float tau, float scale) {
+    float x = __fdiv_rn(tau, scale);
+    if (!(x == x)) return x;  // NaN threshold: nothing compares >= it
+    for (int i = 0; i < 4 && __fmul_rn(x, scale) >= tau; ++i) {
+        const float below = nextafterf(x, -kInf);
+        if (__fmul_rn(below, scale) < tau) break;
+        x = below;
+    }
+    for (int i = 0; i < 4 && __fmul_rn(x, scale) < tau; ++i) x = nextafterf(x, kInf);
+    return x;
+}
+
 }  // namespace saga

@@ -377,6 +377,18 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
     return cuda_status(launch_radix_select(r, s));
 }
 
+// Many records per row (few rows, many slots): several CTAs per row merge
+// shares of about 64 records into partial records stored past the inputs.
+static void set_combine_chunks(const Geometry& g, CombineArgs* ca, void* ws, const WsLayout& L) {
+    const int r_max = max_slots(g, static_cast<long long>(g.b) * g.tiles, ca->C) * ca->recs_per_slot;
+    const int chunks = r_max > 128 ? std::min(32, (r_max + 63) / 64) : 1;
+    if (chunks > 1 && r_max + chunks <= g.S_cap * g.WPK) {
+        ca->chunks = chunks;
+        ca->partial_slot = r_max;
+        ca->tickets = ws_at<uint32_t>(ws, L.tickets);
+    }
+}
+
 // One decode step; the merged rows go to out (normalised), or with part to
 // part as unnormalised per-row records (a sequence shard's contribution).
 static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k, const void* v,
@@ -661,15 +673,7 @@ int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const
     ca.recs_per_slot = g.WPK;
     ca.records = a.records;
     ca.out = out;
-    // Many records per row (few rows, many slots): several CTAs per row merge
-    // shares of about 64 records into partial records stored past the inputs.
-    const int r_max = max_slots(g, static_cast<long long>(g.b) * g.tiles, a.C) * g.WPK;
-    const int chunks = r_max > 128 ? std::min(32, (r_max + 63) / 64) : 1;
-    if (chunks > 1 && r_max + chunks <= g.S_cap * g.WPK) {
-        ca.chunks = chunks;
-        ca.partial_slot = r_max;
-        ca.tickets = ws_at<uint32_t>(ws, L.tickets);
-    }
+    set_combine_chunks(g, &ca, ws, L);
     g_launches += 1;
     return cuda_status(launch_combine(ca, s));
 }
