@@ -186,11 +186,17 @@ def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
 
 # ------------------------------------------------------------------ CPU oracle
 
+def host_cores() -> int:
+    """Host cores this process may run on; the oracle is given as many threads."""
+    return len(os.sched_getaffinity(0))
+
+
 def oracle_sample_us_per_step(w, seed, steps_sample, t0):
     """Times the CPU oracle on one batch element for `steps_sample` steps
     starting at step t0 (refresh steps included as the schedule says) and
     scales to the whole batch.  Returns (us_per_step, cores, description)."""
     import oracle  # test infrastructure: only this leg of the benchmark runs it
+    oracle.set_num_threads(host_cores())
     ws = w.scaled(batch=1)
     K, V = make_cache(ws, seed)
     qs = make_queries(ws, seed, steps=t0 + steps_sample)
@@ -238,13 +244,36 @@ def oracle_single_thread_us(w, seed, t0):
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, world, rank):
+    """The oracle as it stands on the host cores, on the whole batch of the
+    workload: steps W, W+1, ... each timed on its own (the state entering
+    step W set up first, untimed), as many of the K steps as fit in about
+    two minutes of host time."""
     if rank != 0:
         return 0
+    import oracle  # test infrastructure: the reference arm is the oracle
     w = CONFIGS[args.config]
-    n_sample = max(1, args.steps)
-    # bounded: one batch element per step, at most 64 sampled steps
-    n_sample = min(n_sample, 64)
-    us, cores, desc = oracle_sample_us_per_step(w, args.seed, n_sample, args.warmup)
+    cores = host_cores()
+    oracle.set_num_threads(cores)
+    K, V = make_cache(w, args.seed)
+    qs = make_queries(w, args.seed, steps=args.warmup + args.steps)
+    Kh, Vh = bf16_bits(K), bf16_bits(V)
+    del K, V
+    tau = np.full((w.batch, w.h_q), np.nan, np.float32)
+    t_last = (args.warmup // w.n) * w.n
+    if t_last < args.warmup:
+        oracle.atopn_step(bf16_bits(qs[t_last]), Kh, Vh, tau, w.N, t_last, w.n)
+    times, budget_s = [], 120.0
+    for t in range(args.warmup, args.warmup + args.steps):
+        a = time.perf_counter()
+        oracle.atopn_step(bf16_bits(qs[t]), Kh, Vh, tau, w.N, t, w.n)
+        times.append(time.perf_counter() - a)
+        if sum(times) > budget_s:
+            break
+    us = float(np.mean(times)) * 1e6
+    refreshes = sum(1 for t in range(args.warmup, args.warmup + len(times)) if t % w.n == 0)
+    desc = (f"oracle steps {args.warmup}..{args.warmup + len(times) - 1} ({len(times)} of the "
+            f"{args.steps} requested, {refreshes} refresh) on the whole batch ({w.batch} x {w.h_q} "
+            f"rows, l_kv={w.l_kv}), each step timed on its own")
     line = {
         "impl": "reference", "metric": METRIC, "value": us, "unit": "us/step",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -253,10 +282,13 @@ def run_reference(args, world, rank):
         "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_k": w.h_k,
                    "h_v": w.h_v, "head_dim": w.head_dim, "v_head_dim": w.dv, "l_kv": w.l_kv,
                    "N": w.N, "n": w.n,
-                   "parallelism": "replicas" if args.gpus > 1 else "single"},
+                   "parallelism": "replicas" if args.gpus > 1 else "single",
+                   "l2": "host memory (the oracle runs on the CPU)",
+                   "timing": "time.perf_counter around each oracle step, mean over the timed steps"},
         "cpu_baseline": {"value": us, "unit": "us/step", "cores": cores, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "timed_steps": len(times),
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -284,8 +316,12 @@ def run_ours(args, world, rank, local):
     w = CONFIGS[args.config]
     seed = args.seed + rank
     total_steps = args.warmup + args.steps
+    # the end-to-end loop runs whole refresh periods: from the first refresh
+    # step at or after W, as many periods as cover K steps
+    e2e_t0 = -(-args.warmup // w.n) * w.n
+    e2e_steps = -(-args.steps // w.n) * w.n
     K, V = make_cache(w, seed, "cuda")
-    qs = make_queries(w, seed, "cuda", steps=total_steps)
+    qs = make_queries(w, seed, "cuda", steps=max(total_steps, e2e_t0 + e2e_steps))
     dec = AtopNDecoder.for_workload(w)
     stream = torch.cuda.Stream()
     # the inputs and the decoder's zeroed workspace were made on the default
@@ -355,6 +391,7 @@ def run_ours(args, world, rank, local):
             dec.refresh(qs[t_open], K)
         stream.synchronize()
 
+    dec.empty_rows(stream)  # clears the count of the untimed replays
     sampler = ClockSampler(local)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -379,7 +416,8 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(ms, world)
-    us_per_step = ms * 1e3 / args.steps
+    us_window = ms * 1e3 / args.steps
+    empty_rows = dec.empty_rows(stream)
     assert dec.error() == _lib.SAGA_OK
 
     # ---- separately timed step kinds (CUDA-graph replays like the timed
@@ -414,7 +452,11 @@ def run_ours(args, world, rank, local):
     us_refresh = time_steps(lambda r: dec.step(0, qs[0], K, V), 5)
     us_dense = (time_steps(lambda r: dec.dense(qs[r % 4], K, V, out=dense_out), 10)
                 if has_dense else None)
-    us_mix = (us_refresh + (w.n - 1) * us_reuse) / w.n
+    # The headline: one refresh step and n - 1 reuse steps per n tokens, as
+    # the schedule runs them (the K-step window above holds however many
+    # refreshes its position in the period gives it)
+    us_mix = max_over_ranks((us_refresh + (w.n - 1) * us_reuse) / w.n, world)
+    us_per_step = us_mix
 
     # Dense grouped-query attention of the layer SAGA was converted from
     # (h_k = h_v): the pages' full-attention baseline.  Its own cache (more
@@ -472,7 +514,7 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through the public API with host buffers
     q_host = qs.cpu().pin_memory()
-    out_host = torch.empty((args.steps,) + tuple(dec.out.shape), dtype=torch.float32).pin_memory()
+    out_host = torch.empty((e2e_steps,) + tuple(dec.out.shape), dtype=torch.float32).pin_memory()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     barrier(world)
@@ -484,7 +526,7 @@ def run_ours(args, world, rank, local):
         # double buffers, overlapping the neighbouring steps' kernels)
         # The thresholds entering step W (the refresh that opened its period)
         # are put in place outside the timed region before each replay.
-        loop = dec.host_loop(K, V, q_host, out_host, args.warmup, args.steps, stream=stream,
+        loop = dec.host_loop(K, V, q_host, out_host, e2e_t0, e2e_steps, stream=stream,
                              restore=False)
         loop.restore_state()
         loop.replay()             # untimed: the first launch uploads the graph
@@ -500,8 +542,8 @@ def run_ours(args, world, rank, local):
     else:
         # cold like the timed loop above: one host loop of one step per step,
         # L2 flushed before every step outside the events
-        loops = [dec.host_loop(K, V, q_host, out_host[k:k + 1], args.warmup + k, 1, stream=stream,
-                               restore=False) for k in range(args.steps)]
+        loops = [dec.host_loop(K, V, q_host, out_host[k:k + 1], e2e_t0 + k, 1, stream=stream,
+                               restore=False) for k in range(e2e_steps)]
         loops[0].restore_state()  # each later step follows its predecessor
         for lp in loops:          # untimed first launches, in step order
             lp.replay()
@@ -518,12 +560,12 @@ def run_ours(args, world, rank, local):
             e2e_ms += e0.elapsed_time(e1)
         del loops
     barrier(world)
-    e2e_us = max_over_ranks(e2e_ms * 1e3 / args.steps, world)
+    e2e_us = max_over_ranks(e2e_ms * 1e3 / e2e_steps, world)
     # Each step's own output reached the host: the last two steps (one per
     # buffer), recomputed now from the same thresholds, equal it bit for bit
     # (checked when both are reuse steps after the same refresh).
-    last = [(k, args.warmup + k) for k in (args.steps - 2, args.steps - 1)]
-    if args.steps >= 2 and all(t % w.n for _, t in last) and last[0][1] // w.n == last[1][1] // w.n:
+    last = [(k, e2e_t0 + k) for k in (e2e_steps - 2, e2e_steps - 1)]
+    if e2e_steps >= 2 and all(t % w.n for _, t in last) and last[0][1] // w.n == last[1][1] // w.n:
         with torch.cuda.stream(stream):
             for k, t in last:
                 o = dec.step(t, qs[t], K, V).cpu()
@@ -568,6 +610,15 @@ def run_ours(args, world, rank, local):
                    "timing": ("one CUDA-graph replay of K steps, CUDA events" if not cold
                               else "one CUDA graph per step, CUDA events around each replay, "
                                    "summed over K steps")},
+        "value_from": ("one refresh step and n - 1 reuse steps per n tokens, each kind timed as "
+                       "CUDA-graph replays (us_refresh_step, us_reuse_step)"),
+        "window": {"us_per_step": us_window, "steps": args.steps, "first_step": args.warmup,
+                   "refresh_steps": refresh_steps,
+                   "what": "the K timed steps W..W+K-1 as one replay (or one replay per step, cold)"},
+        "empty_set_rows": {"total": int(empty_rows), "steps": args.steps,
+                           "per_step": empty_rows / args.steps,
+                           "what": "rows whose threshold lay above every logit (the empty-set rule "
+                                   "kept their maxima), counted by the library over the K timed steps"},
         "refresh_steps": refresh_steps,
         "gpu_launches": int(gpu_launches),
         "us_reuse_step": us_reuse, "us_refresh_step": us_refresh,
@@ -599,11 +650,14 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": e2e_us, "unit": "us/step",
                 "h2d_bytes_per_step": int(qs[0].numel() * 2),
                 "d2h_bytes_per_step": int(dec.out.numel() * 4),
-                "timing": ("one CUDA-graph replay of the K steps, each with its own copies in "
-                           "and out of pinned host memory on two copy streams (double buffers, "
-                           "overlapping the neighbouring steps' kernels)") if not cold else
-                          "one host loop (CUDA graph) per step with its copies, CUDA events "
-                          "around each replay, L2 flushed before each"},
+                "steps": e2e_steps, "first_step": e2e_t0,
+                "timing": ("whole refresh periods (steps from the first refresh step at or after W, "
+                           "K rounded up to a multiple of n) as one CUDA-graph replay, each step with "
+                           "its own copies in and out of pinned host memory on two copy streams "
+                           "(double buffers, overlapping the neighbouring steps' kernels)") if not cold
+                          else ("whole refresh periods (as above), one host loop (CUDA graph) per step "
+                                "with its copies, CUDA events around each replay, L2 flushed before "
+                                "each")},
         "clocks": sampler.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:

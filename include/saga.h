@@ -32,10 +32,15 @@
  * style head layout, Main Findings "Head count beats head dimension");
  * h_k in {1, 2, 4, 8}; h_q a
  * multiple of h_k and of h_v with h_q/h_k <= 16 and h_q <= 128;
- * saga_decode_dense also needs h_v <= 2*h_k with h_v a multiple or a
- * divisor of h_k, and a stage (32 KB of keys and the value rows of the
- * same positions) that fits twice in shared memory; 1 <= l_kv <= l_cap;
- * batch*l_cap < 2^31.  Others return SAGA_ERR_UNSUPPORTED.
+ * saga_decode_dense also needs h_v a multiple or a divisor of h_k, and a
+ * stage (32 KB of keys and the value rows of the same positions) that fits
+ * twice in shared memory; with more than two value heads per key head, or
+ * a stage too large (e.g. SAGA's (h_k, h_v) = (1, 8), the Sigma-style 32-dim
+ * keys with h_v = 8), the kernel treats every value head as a key head of
+ * its own, each reading its key head's rows (h_v in {2, 4, 8} and
+ * h_q/h_v <= 16 then);
+ * 1 <= l_kv <= l_cap; batch*l_cap < 2^31.  Others return
+ * SAGA_ERR_UNSUPPORTED.
  *
  * Conventions shared by every call:
  *   - Ownership: the caller allocates and owns every buffer (device memory,
@@ -98,7 +103,9 @@ typedef enum {
     SAGA_ERR_WORKSPACE = -3,    /* ws_bytes < saga_workspace_bytes(...) */
     SAGA_ERR_CUDA = -4,         /* a CUDA call or launch failed */
     SAGA_ERR_DEVICE = -5,       /* no device, or the device is not sm_100 */
-    SAGA_ERR_TIMEOUT = -6       /* saga_workspace_error: a bounded device wait ran out */
+    SAGA_ERR_TIMEOUT = -6,      /* saga_workspace_error: a bounded device wait ran out */
+    SAGA_ERR_BOUNDS = -7        /* saga_workspace_error, debug builds (SAGA_DEBUG): a kernel read
+                                   a position, count or slot out of range and skipped it */
 } saga_status;
 
 /* Bytes of workspace the calls below need for these dimensions.  Depends on
@@ -158,6 +165,28 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
                       const float* thresh, const float* logits_in, float* out,
                       int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
                       saga_stream_t stream);
+
+/* One refresh step in one call: the exact thresholds (as
+ * saga_topn_refresh), then the decode with them (as saga_atopn_decode over
+ * the step's logits) -- the step that Atop-N takes on every n-th token
+ * (ai.info summary, Key Contributions #2: the exact top-N threshold is
+ * recomputed, then entries are kept by a per-element comparison).  Results,
+ * bit for bit: thresh_out as saga_topn_refresh writes it; out, sel_idx and
+ * sel_cnt as saga_atopn_decode over those logits writes them.
+ * The logits are written to the workspace once and read twice (the radix
+ * passes of the threshold's first two digits): the second also copies out
+ * every logit at or above the lower edge of the threshold's first-digit
+ * bucket (every kept one among them), and one kernel then finds the last
+ * digit and compacts the kept entries from those candidates alone.  Exceptions: N >= l_kv (thresh_out = -inf, full attention) and
+ * rows longer than the compaction's on-chip bitmap allows (l_kv above about
+ * 900K) compact from the stored logits; few long rows (b*h_q <= 64 and
+ * l_kv >= 65536) take saga_atopn_decode's fused path after the refresh (the
+ * same logits, recomputed bit for bit).
+ * q, k, v, thresh_out [b,h_q], out [b,h_q,d_v]: required.
+ * sel_idx, sel_cnt (nullable): as in saga_atopn_decode. */
+int saga_atopn_refresh_step(const saga_dims* dims, int32_t N, const void* q, const void* k,
+                            const void* v, float* thresh_out, float* out, int32_t* sel_idx,
+                            int32_t* sel_cnt, void* ws, size_t ws_bytes, saga_stream_t stream);
 
 /* ---- Sequence shards (the pages run one GPU; this is an extension) ----
  * A decode whose cached sequence is split into contiguous shards, one per
@@ -265,8 +294,19 @@ int saga_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us, sag
 int saga_workspace_reset(void* ws, size_t ws_bytes, saga_stream_t stream);
 
 /* Synchronise `stream`, read and clear the workspace's sticky device flag:
- * SAGA_OK, SAGA_ERR_TIMEOUT, or SAGA_ERR_CUDA if the read itself failed. */
+ * SAGA_OK, SAGA_ERR_TIMEOUT, SAGA_ERR_BOUNDS (debug builds only: the
+ * library compiled with SAGA_DEBUG checks every position, count and slot a
+ * kernel takes from another kernel's output, and skips the access instead
+ * of trapping), or SAGA_ERR_CUDA if the read itself failed. */
 int saga_workspace_error(void* ws, size_t ws_bytes, saga_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the workspace's count of rows
+ * that kept nothing and took the empty-set rule (tau_eff = min(tau, row
+ * max): a stale threshold above every logit of the row keeps its maximal
+ * entries; the pages leave that case open) in the decode calls since the
+ * last read, into *count_out.  Rows of saga_atopn_decode_partial are not
+ * counted (the merge of the shards decides their rule). */
+int saga_workspace_empty_rows(void* ws, size_t ws_bytes, uint64_t* count_out, saga_stream_t stream);
 
 /* Static description of a status code. */
 const char* saga_status_string(int status);

@@ -13,7 +13,11 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIBRARY = os.path.join(_HERE, "libsaga.so")
+# The bounds-checked build (SAGA_DEBUG) sits beside the release one; the
+# SAGA_LIBRARY environment variable picks the library a process loads.
+RELEASE_LIBRARY = os.path.join(_HERE, "libsaga.so")
+DEBUG_LIBRARY = os.path.join(_HERE, "libsaga_debug.so")
+LIBRARY = os.environ.get("SAGA_LIBRARY") or RELEASE_LIBRARY
 
 SAGA_OK = 0
 SAGA_ERR_INVALID_ARG = -1
@@ -22,6 +26,7 @@ SAGA_ERR_WORKSPACE = -3
 SAGA_ERR_CUDA = -4
 SAGA_ERR_DEVICE = -5
 SAGA_ERR_TIMEOUT = -6
+SAGA_ERR_BOUNDS = -7
 
 EXPORTS = (
     "saga_workspace_bytes", "saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
@@ -29,6 +34,7 @@ EXPORTS = (
     "saga_set_kernel_events", "saga_version", "saga_topn_refresh_noalloc",
     "saga_selftest_wait_timeout", "saga_cache_append", "saga_qk_logits", "saga_topn_histogram",
     "saga_topn_select_digit", "saga_atopn_decode_partial", "saga_merge_partials",
+    "saga_atopn_refresh_step", "saga_workspace_empty_rows",
 )
 
 
@@ -66,6 +72,7 @@ def load(path: str | None = None):
         lib.saga_decode_dense.argtypes = [D, P, P, P, P, P, SZ, P]
         lib.saga_topn_refresh.argtypes = [D, I32, P, P, P, P, P, P, SZ, P]
         lib.saga_atopn_decode.argtypes = [D, P, P, P, P, P, P, P, P, P, SZ, P]
+        lib.saga_atopn_refresh_step.argtypes = [D, I32, P, P, P, P, P, P, P, P, SZ, P]
         lib.saga_topn_refresh_noalloc.argtypes = [D, I32, P, P, P]
         lib.saga_topn_refresh_noalloc.restype = ctypes.c_int
         lib.saga_cache_append.argtypes = [D, P, P, P, P, P]
@@ -74,6 +81,8 @@ def load(path: str | None = None):
         lib.saga_selftest_wait_timeout.restype = ctypes.c_int
         lib.saga_workspace_reset.argtypes = [P, SZ, P]
         lib.saga_workspace_error.argtypes = [P, SZ, P]
+        lib.saga_workspace_empty_rows.argtypes = [P, SZ, ctypes.POINTER(ctypes.c_uint64), P]
+        lib.saga_workspace_empty_rows.restype = ctypes.c_int
         lib.saga_status_string.argtypes = [ctypes.c_int]
         lib.saga_status_string.restype = ctypes.c_char_p
         lib.saga_launch_count.restype = ctypes.c_uint64
@@ -84,7 +93,7 @@ def load(path: str | None = None):
         lib.saga_topn_select_digit.argtypes = [D, I32, I32, P, P, P, P]
         lib.saga_atopn_decode_partial.argtypes = [D, P, P, P, P, P, P, P, SZ, P]
         lib.saga_merge_partials.argtypes = [D, P, I32, P, P, P]
-        for f in ("saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode",
+        for f in ("saga_decode_dense", "saga_topn_refresh", "saga_atopn_decode", "saga_atopn_refresh_step",
                   "saga_workspace_reset", "saga_workspace_error", "saga_version", "saga_qk_logits",
                   "saga_topn_histogram", "saga_topn_select_digit", "saga_atopn_decode_partial",
                   "saga_merge_partials"):
@@ -184,6 +193,13 @@ def topn_select_digit(d, N: int, pass_: int, hist, state, thresh_out, stream=Non
                                          _ptr(state), _ptr(thresh_out), _stream(stream)))
 
 
+def atopn_refresh_step(d, N, q, k, v, thresh_out, out, sel_idx, sel_cnt, ws, stream=None) -> None:
+    st = load().saga_atopn_refresh_step(ctypes.byref(d), int(N), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(thresh_out), _ptr(out), _ptr(sel_idx), _ptr(sel_cnt),
+                                        _ptr(ws), ws.numel() * ws.element_size(), _stream(stream))
+    _check("saga_atopn_refresh_step", st)
+
+
 def atopn_decode_partial(d, q, k, v, thresh, logits_in, part, ws, stream=None) -> None:
     _check("saga_atopn_decode_partial",
            load().saga_atopn_decode_partial(ctypes.byref(d), _ptr(q), _ptr(k), _ptr(v),
@@ -212,6 +228,15 @@ def workspace_reset(ws, stream=None) -> None:
 def workspace_error(ws, stream=None) -> int:
     return int(load().saga_workspace_error(_ptr(ws), ws.numel() * ws.element_size(),
                                            _stream(stream)))
+
+
+def workspace_empty_rows(ws, stream=None) -> int:
+    """Rows that took the empty-set rule since the last read (read and cleared)."""
+    n = ctypes.c_uint64(0)
+    _check("saga_workspace_empty_rows",
+           load().saga_workspace_empty_rows(_ptr(ws), ws.numel() * ws.element_size(), ctypes.byref(n),
+                                            _stream(stream)))
+    return int(n.value)
 
 
 def launch_count() -> int:

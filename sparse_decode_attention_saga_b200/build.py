@@ -1,10 +1,14 @@
 """Builds ``libsaga.so`` (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m sparse_decode_attention_saga_b200.build [--force] [--verbose]
+    python -m sparse_decode_attention_saga_b200.build [--force] [--verbose] [--debug]
 
 Each ``csrc/*.cu`` file is compiled to an object under ``_build/`` (in
 parallel), then linked into ``sparse_decode_attention_saga_b200/libsaga.so``.
-Objects are rebuilt when their source or any header is newer.
+Objects are rebuilt when their source or any header is newer.  ``--debug``
+builds ``libsaga_debug.so`` instead (objects under ``_build/debug/``), with
+SAGA_DEBUG defined: every position, count and slot a kernel reads from
+another kernel's output is bounds-checked, an out-of-range one sets a sticky
+error bit and is skipped.
 """
 from __future__ import annotations
 
@@ -22,6 +26,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIBRARY = os.path.join(PKG, "libsaga.so")
+DEBUG_LIBRARY = os.path.join(PKG, "libsaga_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
@@ -40,14 +45,18 @@ def _headers():
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: bool = False) -> str:
     nvcc = _nvcc()
-    os.makedirs(BUILD, exist_ok=True)
+    build_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    library = DEBUG_LIBRARY if debug else LIBRARY
+    if debug:
+        extra_flags = tuple(extra_flags) + ("-DSAGA_DEBUG=1",)
+    os.makedirs(build_dir, exist_ok=True)
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     newest_header = max((os.path.getmtime(h) for h in _headers()), default=0.0)
     objects, jobs = [], []
     for src in sources:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objects.append(obj)
         if force or not os.path.exists(obj) or \
                 os.path.getmtime(obj) < max(os.path.getmtime(src), newest_header):
@@ -69,19 +78,20 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
                 failed.append(cmd[-3])
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(failed))
-    if jobs or force or not os.path.exists(LIBRARY):
-        tmp = LIBRARY + ".tmp"
+    if jobs or force or not os.path.exists(library):
+        tmp = library + ".tmp"
         cmd = [nvcc] + ARCH + ["-shared", "-o", tmp] + objects
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode:
             raise RuntimeError("link failed:\n" + r.stdout + r.stderr)
-        os.replace(tmp, LIBRARY)
-    return LIBRARY
+        os.replace(tmp, library)
+    return library
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose))
+    print(build(force=a.force, verbose=a.verbose, debug=a.debug))

@@ -155,9 +155,11 @@ __device__ void combine_row(const CombineArgs& a, long long row, int r_begin = 0
 
     float* out_row = a.out + static_cast<size_t>(row) * D;
     if (cnt == 0 && a.fallback && !partial_out) {
-        if (warp == 0)
+        if (warp == 0) {
             fallback_row<D, DK, NT>(a, row, mall, out_row, a.sel_cnt ? a.sel_cnt + row : nullptr, kbuf,
                                     false, a.sel_idx ? a.sel_idx + static_cast<size_t>(row) * g.l : nullptr);
+            if (lane == 0 && a.empty_rows) atomicAdd(a.empty_rows, 1u);
+        }
         return;
     }
 
@@ -297,6 +299,7 @@ __device__ void merge_same_reference(const CombineArgs& a, long long row, int R,
                     part[2] = __int_as_float(0);
                     part[3] = m_all;
                 }
+                if (!part && lane == 0 && a.empty_rows) atomicAdd(a.empty_rows, 1u);
             }
         } else {
             for (int k = tid; k < D; k += kCombineThreads) out_row[k] = 0.f;

@@ -17,6 +17,11 @@
 //   registers.  The query heads of one column tile share one value head.
 // Every warp writes one partial record per (row, CTA slot); the combine
 // kernel merges them.
+// More than two value heads per key head (SAGA's (h_k, h_v) = (1, 8), or
+// 32-dim keys with h_v = 4 h_k): the kernel runs on a geometry with one key
+// head per value head, each loading its cache key head (k_group of them
+// share one), so that every warp's query heads use a single value head.
+// The shared key rows then come from HBM once and from L2 k_group times.
 #include "qk_tile.cuh"
 #include "saga_kernels.h"
 
@@ -86,7 +91,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 for (int kh = 0; kh < g.hk; ++kh)
                     for (int dh = 0; dh < KTile<D>::NBOX; ++dh)
                         tma_load_3d(dst + (kh * KTile<D>::NBOX + dh) * g.P * KTile<D>::ROWB, &kmap,
-                                    &full[st], dh * 64, kh, z);
+                                    &full[st], dh * 64, kh / a.k_group, z);
                 for (int vh = 0; vh < g.hv; ++vh)
                     for (int dh = 0; dh < DVH; ++dh)
                         tma_load_3d(dst + kStageBytes + (vh * DVH + dh) * g.P * 128, &vmap,

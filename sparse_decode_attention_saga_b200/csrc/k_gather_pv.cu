@@ -80,7 +80,9 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
     if (a.mode == kListContiguous) {
         if (tid == 0) {
             pre[0] = 0;
-            pre[1] = min(max(__ldg(a.cnt + row), 0), g.l);
+            const int c = __ldg(a.cnt + row);
+            in_bounds(c >= 0 && c <= g.l, a.err);
+            pre[1] = min(max(c, 0), g.l);
             start[0] = 0;
             row_base = row * g.l;
         }
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
                         sl_prev = sl;
                     }
                     start[j] = pos + (j - sl * g.WPK) * cap;
+                    in_bounds(cu[u] >= 0 && cu[u] <= cap, a.err);
                     const int cnt_j = cu[u] < 0 ? 0 : (cu[u] > cap ? cap : cu[u]);
                     pre[j] = cnt_j;
                     run += cnt_j;
@@ -219,6 +222,10 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
                 const int2 ps = __ldg(a.seg_list + at);
                 pos = ps.x;
                 s = __int_as_float(ps.y);
+            }
+            if (!in_bounds(pos >= 0 && pos < g.l, a.err)) {
+                pos = 0;
+                s = -kInf;
             }
         }
     };

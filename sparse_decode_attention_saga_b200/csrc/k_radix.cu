@@ -15,9 +15,14 @@
 // from the top bin, fixes the digit that holds the rank, and stores
 // (prefix, rank) for the next pass, or the threshold after the last pass.
 // No CTA waits for another.  With a candidate buffer, pass 1 also copies the
-// logits of its prefix bucket into its chunk's part of the buffer (one
-// shared-memory counter per CTA, reserved a warp at a time), and pass 2 reads
-// only those candidates, each CTA its own chunk's.
+// (position, logit) of every key at or above the lower edge of pass 0's
+// bucket into its chunk's part of the buffer (one shared-memory counter per
+// CTA; the order inside a chunk is not fixed), and pass 2 reads only those
+// candidates, each CTA its own chunk's.  The kept set (logit >= threshold)
+// lies among them, so the ordered compaction can read them instead of the
+// logits (k_select.cu).
+#include <type_traits>
+
 #include "saga_device.cuh"
 #include "saga_kernels.h"
 
@@ -55,7 +60,8 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t& e
 // counts on them (the scalar path keeps its registers).
 template <int PASS, int VEC>
 __global__ void __launch_bounds__(kThreads, VEC == 4 ? 8 : 4) radix_pass_kernel(const RadixArgs a) {
-    constexpr int kLoadsV = kLoads / VEC;  // VEC-wide loads per thread per round
+    constexpr int kLoadsV = kLoads / VEC;        // VEC-wide loads per thread per round
+    constexpr int kRound = kLoads * kThreads;    // positions per round
     constexpr int shift = PASS == 0 ? 21 : (PASS == 1 ? 10 : 0);
     constexpr int width = PASS == 2 ? 10 : 11;
     constexpr int nb = 1 << width;
@@ -76,75 +82,99 @@ __global__ void __launch_bounds__(kThreads, VEC == 4 ? 8 : 4) radix_pass_kernel(
     if (tid == 0) s_cand = 0;
     const uint32_t prefix = PASS == 0 ? 0u : __ldcg(a.state + row * 2);
     __syncthreads();
-    const int lane = tid & 31;
     const bool from_cand = PASS == 2 && a.cand != nullptr;
 
     const float* src = a.logits + row * a.l;
-    const int per = ((a.l + a.chunks - 1) / a.chunks + 3) & ~3;  // multiple of 4
+    const int per = radix_chunk_len(a.l, a.chunks);
     const int j0 = from_cand ? 0 : chunk * per;
     const int j1 = from_cand ? 0 : min(a.l, j0 + per);
-    float* cdst = PASS == 1 && a.cand ? a.cand + row * a.l + static_cast<long long>(chunk) * per : nullptr;
+    int2* cdst = PASS == 1 && a.cand ? a.cand + row * a.l + static_cast<long long>(chunk) * per : nullptr;
+    // pass 1 copies out every logit at or above the lower edge of pass 0's
+    // bucket: the bucket's members (pass 2 reads them) and every larger
+    // one, so that the kept set (logit >= threshold) lies among them.
+    // The test is a float compare against the bucket's lower edge (the
+    // order of the keys is the order of the floats), so that the key is
+    // computed for members only.  The lowest buckets (-inf and negative
+    // NaNs) have a NaN for an edge: every logit is a member then, a superset
+    // that pass 2 and the compaction filter.  (Logits are finite: a NaN
+    // would take its key's place in pass 0 but not in this compare.)
+    const float lo_f = key_to_float(prefix << 21);
+    const bool all_members = isnan(lo_f);
+    // the member's key into the histogram (its bucket's next digit) and, with
+    // a candidate buffer, its (position, logit) into this chunk's part
+    auto member = [&](float x, int j) {
+        const uint32_t key = float_to_key(x);
+        if ((key >> high) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+        if (cdst) cdst[atomicAdd(&s_cand, 1)] = make_int2(j, __float_as_int(x));
+    };
     // 64 bytes of independent coalesced loads per thread per round (16-byte
     // loads when the rows are 16-byte aligned) keep enough bytes in flight to
-    // stream the logits at HBM speed.
-    for (int base = j0; base < j1; base += kLoadsV * kThreads * VEC) {
+    // stream the logits at HBM speed; whole rounds skip the bounds checks.
+    auto round = [&](int base, auto whole) {
+        constexpr bool kWhole = decltype(whole)::value;
         float v[kLoadsV][VEC];
 #pragma unroll
         for (int k = 0; k < kLoadsV; ++k) {
             const int j = base + (k * kThreads + tid) * VEC;
-            if (VEC == 4 && j + VEC <= j1) {
+            if (VEC == 4 && (kWhole || j + VEC <= j1)) {
                 const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
                 const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                 for (int c = 0; c < VEC; ++c) v[k][c] = xs[c];
             } else {
 #pragma unroll
-                for (int c = 0; c < VEC; ++c) v[k][c] = j + c < j1 ? __ldg(src + j + c) : 0.f;
+                for (int c = 0; c < VEC; ++c) v[k][c] = kWhole || j + c < j1 ? __ldg(src + j + c) : 0.f;
             }
         }
-        uint32_t cm = 0u;  // pass 1: which of this round's values are bucket members
+        if constexpr (PASS == 1) {
+            // Members are a few percent of the logits: a bitmask of this
+            // thread's members (branch-free), then one short loop over the
+            // set bits, each member's logit read again from L1.
+            uint32_t m = 0u;
 #pragma unroll
-        for (int k = 0; k < kLoadsV; ++k) {
+            for (int k = 0; k < kLoadsV; ++k)
 #pragma unroll
-            for (int c = 0; c < VEC; ++c) {
-                const int j = base + (k * kThreads + tid) * VEC + c;
-                const uint32_t key = float_to_key(v[k][c]);
-                const bool cand = j < j1 && (PASS == 0 || (key >> high) == prefix);
-                if (cand) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-                if (PASS == 1 && cand) cm |= 1u << (k * VEC + c);
+                for (int c = 0; c < VEC; ++c) {
+                    const int j = base + (k * kThreads + tid) * VEC + c;
+                    const bool in = (kWhole || j < j1) && (v[k][c] >= lo_f || all_members);
+                    m |= static_cast<uint32_t>(in) << (k * VEC + c);
+                }
+            while (m) {
+                const int e = __ffs(m) - 1;
+                m &= m - 1u;
+                const int j = base + ((e / VEC) * kThreads + tid) * VEC + e % VEC;
+                member(__ldg(src + j), j);
             }
+        } else {
+#pragma unroll
+            for (int k = 0; k < kLoadsV; ++k)
+#pragma unroll
+                for (int c = 0; c < VEC; ++c) {
+                    const int j = base + (k * kThreads + tid) * VEC + c;
+                    if (kWhole || j < j1) {
+                        const uint32_t key = float_to_key(v[k][c]);
+                        if (PASS == 0) {
+                            atomicAdd(&hist[key >> shift], 1u);
+                        } else if ((key >> high) == prefix) {
+                            atomicAdd(&hist[key & (nb - 1)], 1u);
+                        }
+                    }
+                }
         }
-        if (PASS == 1 && cdst) {
-            // copy this round's bucket members out: a warp-wide scan of the
-            // per-thread counts, one shared-memory reservation per warp
-            const int mine = __popc(cm);
-            int inc = mine;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int x = __shfl_up_sync(0xffffffffu, inc, o);
-                if (lane >= o) inc += x;
-            }
-            const int wtot = __shfl_sync(0xffffffffu, inc, 31);
-            if (wtot > 0) {
-                int wbase = 0;
-                if (lane == 31) wbase = atomicAdd(&s_cand, wtot);
-                wbase = __shfl_sync(0xffffffffu, wbase, 31);
-                int at = wbase + inc - mine;
-#pragma unroll
-                for (int k = 0; k < kLoadsV; ++k)
-#pragma unroll
-                    for (int c = 0; c < VEC; ++c)
-                        if (cm & (1u << (k * VEC + c))) cdst[at++] = v[k][c];
-            }
-        }
-    }
-    if (from_cand) {
+    };
+    if (!from_cand) {
+        int base = j0;
+        for (; base + kRound <= j1; base += kRound) round(base, std::true_type{});
+        if (base < j1) round(base, std::false_type{});
+    } else {
         // pass 2 over the candidates pass 1 copied out of this chunk
-        const int n = min(max(__ldcg(a.cand_cnt + row * kRadixMaxChunks + chunk), 0), per);
-        const float* cs = a.cand + row * a.l + static_cast<long long>(chunk) * per;
+        const int nc = __ldcg(a.cand_cnt + row * kRadixMaxChunks + chunk);
+        in_bounds(nc >= 0 && nc <= per, a.err);
+        const int n = min(max(nc, 0), per);
+        const int2* cs = a.cand + row * a.l + static_cast<long long>(chunk) * per;
         for (int j = tid; j < n; j += kThreads) {
-            const uint32_t key = float_to_key(__ldcg(cs + j));
-            if ((key >> high) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+            const uint32_t key = float_to_key(__int_as_float(__ldcg(cs + j).y));
+            if ((key >> high) == prefix) atomicAdd(&hist[key & (nb - 1)], 1u);
         }
     }
     __syncthreads();
@@ -213,13 +243,15 @@ cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream) {
         radix_pass_kernel<0, 4><<<grid, block, 0, stream>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e == cudaSuccess) e = launch_dependent(radix_pass_kernel<1, 4>, grid, block, 0, stream, a);
-        if (e == cudaSuccess) e = launch_dependent(radix_pass_kernel<2, 4>, grid, block, 0, stream, a);
+        if (e == cudaSuccess && a.passes > 2)
+            e = launch_dependent(radix_pass_kernel<2, 4>, grid, block, 0, stream, a);
         return e;
     }
     radix_pass_kernel<0, 1><<<grid, block, 0, stream>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) e = launch_dependent(radix_pass_kernel<1, 1>, grid, block, 0, stream, a);
-    if (e == cudaSuccess) e = launch_dependent(radix_pass_kernel<2, 1>, grid, block, 0, stream, a);
+    if (e == cudaSuccess && a.passes > 2)
+        e = launch_dependent(radix_pass_kernel<2, 1>, grid, block, 0, stream, a);
     return e;
 }
 

@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
                 const int j = base + (k * kThreads + tid) * VEC;
 #pragma unroll
                 for (int c = 0; c < VEC; ++c) {
-                    if (kb[k] & (1u << c)) {
+                    if ((kb[k] & (1u << c)) && in_bounds(at < a.l, a.err)) {
                         dst[at] = j + c;
                         sdst[at] = v[k][c];
                         ++at;
@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(kThreads) select_compact_kernel(const SelectAr
             __syncthreads();
         }
         if (total > 0 || !a.keep_max) break;
+        if (tid == 0 && a.empty_rows) atomicAdd(a.empty_rows, 1u);  // the empty-set rule fires
     }
     if (tid == 0) a.cnt[row] = total;
 }
@@ -159,7 +160,9 @@ __global__ void __launch_bounds__(kThreads) lists_to_index_kernel(const IndexArg
     const int32_t* cnt = a.seg_cnt + static_cast<size_t>(row) * g.S_cap * g.WPK;
     auto clamped = [&](int j, SegList& sl) {
         sl = seg_list_of(g.P, g.MBW, g.WPK, g.tiles, bb, j, T, a.C);
-        return min(max(__ldg(cnt + j), 0), sl.cap);
+        const int c = __ldg(cnt + j);
+        in_bounds(c >= 0 && c <= sl.cap, a.err);
+        return min(max(c, 0), sl.cap);
     };
     int mine = 0;
     for (int j = tid; j < nl; j += kThreads) {
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(kThreads) lists_to_index_kernel(const IndexArg
         const int n = clamped(j, sl);
         for (int e = lane; e < n; e += 32) {
             const int pos = __ldg(&lists[sl.start + e].x);
-            if (pos >= 0 && pos < g.l) atomicOr(bm + (pos >> 5), 1u << (pos & 31));
+            if (in_bounds(pos >= 0 && pos < g.l, a.err)) atomicOr(bm + (pos >> 5), 1u << (pos & 31));
         }
     }
     __syncthreads();
@@ -216,7 +219,186 @@ __global__ void __launch_bounds__(kThreads) lists_to_index_kernel(const IndexArg
     }
 }
 
+// One CTA per row over the radix candidates.  With the radix state of the
+// first two digits (a.state), the threshold's last digit comes first: the
+// candidates in the 22-bit prefix bucket are histogrammed by their last 10
+// bits in shared memory and a block scan picks the bin holding the rank
+// still sought, which completes the exact N-th largest logit (written to
+// a.thresh; the third radix pass is not needed).  Then every candidate at or
+// above the threshold sets its position's bit in a shared bitmap (a
+// position is a candidate at most once), each thread takes a contiguous run
+// of bitmap words and a block scan of the runs' counts gives every word's
+// rank, and each kept candidate is written at its word's rank plus the set
+// bits below it, so the output is ascending whatever order the candidates
+// came in.  The row's largest logit is the largest candidate.  Nothing kept
+// (only when the threshold lies above every logit) keeps the row's maxima,
+// as the compaction over stored logits does.
+// Dynamic shared memory (cand_select_smem): bitmap [words] | word ranks [words].
+constexpr int kCandThreads = 512;
+constexpr int kCandWarps = kCandThreads / 32;
+
+__device__ __forceinline__ uint32_t cand_block_scan(uint32_t v, uint32_t& excl, uint32_t* warp_tot) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += x;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kCandWarps; ++w) {
+        before += w < warp ? warp_tot[w] : 0u;
+        total += warp_tot[w];
+    }
+    excl = before + inc - v;
+    return total;
+}
+
+__global__ void __launch_bounds__(kCandThreads) cand_select_kernel(const CandSelectArgs a) {
+    extern __shared__ uint32_t bm[];
+    __shared__ uint32_t warp_tot[kCandWarps];
+    __shared__ float red[kCandWarps];
+    __shared__ uint32_t hist[1024];
+    __shared__ float s_tau;
+    pdl_wait();  // candidates and radix state (or thresholds) from the radix passes
+    pdl_trigger();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const long long row = blockIdx.x;
+    const int words = (a.l + 31) >> 5;
+    uint32_t* wrank = bm + words;
+    const int per = radix_chunk_len(a.l, a.chunks);
+    const int2* cand = a.cand + row * a.l;
+    const int32_t* ccnt = a.cand_cnt + row * kRadixMaxChunks;
+    // every candidate of the row, chunk by chunk: fn(position, logit), four
+    // independent loads per thread in flight
+    auto each = [&](auto fn) {
+        for (int c = 0; c < a.chunks; ++c) {
+            const int nc = __ldcg(ccnt + c);
+            in_bounds(nc >= 0 && nc <= per, a.err);
+            const int n = min(max(nc, 0), per);
+            const int2* cs = cand + static_cast<long long>(c) * per;
+            for (int e0 = 0; e0 < n; e0 += 4 * kCandThreads) {
+                int2 p[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + u * kCandThreads + tid;
+                    p[u] = e < n ? __ldcg(cs + e) : make_int2(-1, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (e0 + u * kCandThreads + tid < n && in_bounds(p[u].x >= 0 && p[u].x < a.l, a.err))
+                        fn(p[u].x, __int_as_float(p[u].y));
+            }
+        }
+    };
+
+    float tau;
+    if (a.state) {
+        // the last 10 bits of the N-th largest key
+        const uint32_t prefix = __ldcg(a.state + row * 2), rank = __ldcg(a.state + row * 2 + 1);
+        for (int i = tid; i < 1024; i += kCandThreads) hist[i] = 0u;
+        __syncthreads();
+        each([&](int, float x) {
+            const uint32_t key = float_to_key(x);
+            if ((key >> 10) == prefix) atomicAdd(&hist[key & 1023u], 1u);
+        });
+        __syncthreads();
+        constexpr int kPer = 1024 / kCandThreads;  // bins per thread, from the top
+        const int top = 1024 - tid * kPer;
+        uint32_t cnt[kPer], sum = 0;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            cnt[k] = hist[top - 1 - k];
+            sum += cnt[k];
+        }
+        uint32_t excl;
+        cand_block_scan(sum, excl, warp_tot);
+        if (excl < rank && rank <= excl + sum) {
+            uint32_t before = excl;
+            int digit = top - 1;
+#pragma unroll
+            for (int k = 0; k < kPer; ++k) {
+                if (before + cnt[k] >= rank) {
+                    digit = top - 1 - k;
+                    break;
+                }
+                before += cnt[k];
+            }
+            const float t = key_to_float((prefix << 10) | static_cast<uint32_t>(digit));
+            s_tau = t;
+            a.thresh[row] = t;
+        }
+        __syncthreads();
+        tau = s_tau;
+    } else {
+        tau = __ldg(a.thresh + row);
+    }
+
+    float m = -kInf;
+    uint32_t total = 0;
+    for (int pass = 0; pass < 2; ++pass) {
+        for (int w = tid; w < words; w += kCandThreads) bm[w] = 0u;
+        __syncthreads();
+        each([&](int pos, float x) {
+            if (pass == 0) m = fmaxf(m, x);
+            if (x >= tau) atomicOr(bm + (pos >> 5), 1u << (pos & 31));
+        });
+        if (pass == 0) {
+            m = warp_max(m);
+            if (lane == 0) red[warp] = m;
+        }
+        __syncthreads();
+        const int run = (words + kCandThreads - 1) / kCandThreads;
+        const int w0 = min(words, tid * run), w1 = min(words, w0 + run);
+        uint32_t c = 0;
+        for (int w = w0; w < w1; ++w) c += __popc(bm[w]);
+        uint32_t at;
+        total = cand_block_scan(c, at, warp_tot);
+        for (int w = w0; w < w1; ++w) {
+            wrank[w] = at;
+            at += __popc(bm[w]);
+        }
+        if (pass == 0) {
+            m = red[0];
+#pragma unroll
+            for (int w = 1; w < kCandWarps; ++w) m = fmaxf(m, red[w]);
+        }
+        if (total > 0) break;
+        tau = m;  // nothing passed: keep the maxima
+        if (tid == 0 && a.empty_rows) atomicAdd(a.empty_rows, 1u);
+        __syncthreads();
+    }
+    __syncthreads();
+    int32_t* dst = a.idx + row * a.l;
+    float* sdst = a.s + row * a.l;
+    each([&](int pos, float x) {
+        const int w = pos >> 5;
+        const uint32_t bits = bm[w], bit = 1u << (pos & 31);
+        if (!(bits & bit)) return;
+        const uint32_t r = wrank[w] + __popc(bits & (bit - 1u));
+        dst[r] = pos;
+        sdst[r] = x;
+    });
+    if (tid == 0) {
+        a.cnt[row] = static_cast<int32_t>(total);
+        a.rowmax[row] = m;
+    }
+}
+
 }  // namespace
+
+size_t cand_select_smem(int l) { return 2 * ((static_cast<size_t>(l) + 31) / 32) * sizeof(uint32_t); }
+
+cudaError_t launch_cand_select(const CandSelectArgs& a, cudaStream_t stream) {
+    const size_t smem = cand_select_smem(a.l);
+    const cudaError_t e = allow_dynamic_smem(cand_select_kernel, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    return launch_dependent(cand_select_kernel, dim3(static_cast<unsigned>(a.rows)), dim3(kCandThreads),
+                            smem, stream, a);
+}
 
 cudaError_t launch_lists_to_index(const IndexArgs& a, cudaStream_t stream) {
     const long long rows = static_cast<long long>(a.g.b) * a.g.hq;

@@ -136,6 +136,23 @@ int make_geometry(const saga_dims* d, Geometry* g) {
     return SAGA_OK;
 }
 
+// The dense kernel's geometry: the cache's own, or, with more than two value
+// heads per key head (or a stage of two that does not fit twice in shared
+// memory), one key head per value head, of which each group of *k_group
+// reads the same cache key head.
+int dense_geometry(const saga_dims* d, Geometry* g, int* k_group) {
+    int st = make_geometry(d, g);
+    *k_group = 1;
+    if (st) return st;
+    if (g->hv <= 2 * g->hk && dense_smem_bytes(*g, 2) <= static_cast<size_t>(kMaxDynamicSmem)) return st;
+    if (g->hv <= g->hk || g->hv % g->hk) return SAGA_ERR_UNSUPPORTED;
+    saga_dims dd = *d;
+    dd.h_k = d->h_v;
+    if ((st = make_geometry(&dd, g))) return st;
+    *k_group = d->h_v / d->h_k;
+    return SAGA_OK;
+}
+
 int check_ws(const Geometry& g, const void* ws, size_t ws_bytes) {
     if (!ws || !aligned(ws, 256)) return SAGA_ERR_INVALID_ARG;
     if (ws_bytes < workspace_layout(g).total) return SAGA_ERR_WORKSPACE;
@@ -281,46 +298,144 @@ namespace saga {
 void note_launches(int n) { g_launches += static_cast<uint64_t>(n); }
 
 namespace {
-// (kernel, limit) pairs whose attribute has been set, with a bit per device.
+// The largest dynamic shared-memory limit set so far for each kernel, per device.
 struct SmemAttr {
     const void* fn;
-    int bytes;
-    uint64_t devices;
+    int bytes[kMaxDevices];
 };
 constexpr int kMaxSmemAttrs = 128;
+constexpr int kDefaultDynamicSmem = 48 * 1024;  // needs no attribute
 SmemAttr g_smem_attr[kMaxSmemAttrs];
 int g_n_smem_attr = 0;
 std::mutex g_smem_attr_mu;
 }  // namespace
 
 cudaError_t allow_dynamic_smem(const void* fn, int bytes) {
+    if (bytes <= kDefaultDynamicSmem) return cudaSuccess;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    const uint64_t bit = 1ull << dev;
     std::lock_guard<std::mutex> lock(g_smem_attr_mu);
     SmemAttr* rec = nullptr;
     for (int i = 0; i < g_n_smem_attr; ++i)
-        if (g_smem_attr[i].fn == fn && g_smem_attr[i].bytes == bytes) rec = &g_smem_attr[i];
-    if (rec && (rec->devices & bit)) return cudaSuccess;
+        if (g_smem_attr[i].fn == fn) rec = &g_smem_attr[i];
+    if (rec && rec->bytes[dev] >= bytes) return cudaSuccess;  // never lowered
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     if (!rec && g_n_smem_attr < kMaxSmemAttrs) {
         rec = &g_smem_attr[g_n_smem_attr++];
-        *rec = SmemAttr{fn, bytes, 0};
+        rec->fn = fn;
+        for (int d = 0; d < kMaxDevices; ++d) rec->bytes[d] = 0;
     }
-    if (rec) rec->devices |= bit;  // (a full table only means setting it again next time)
+    if (rec) rec->bytes[dev] = bytes;  // (a full table only means setting it again next time)
     return cudaSuccess;
 }
 }  // namespace saga
 
+// The workspace header's counter of empty-set rows (the word after the
+// sticky error flag).
+static uint32_t* ws_empty_rows(void* ws, const WsLayout& L) { return ws_at<uint32_t>(ws, L.err) + 1; }
+
+// Exact thresholds over stored logits, or over logits computed here into
+// logits_out (the workspace's logits region when null).  The radix pass 1
+// leaves its candidates (every logit at or above the lower edge of the
+// threshold's first-digit bucket) in the workspace for the compaction of a
+// refresh step (thresholds of -inf and no candidates when N >= l).  With
+// two_digits the passes stop there: the compaction over the candidates
+// finds the last digit and writes the thresholds.
+static int refresh_impl(const Geometry& g, const DeviceInfo& dev, int32_t N, const void* q,
+                        const void* k, const float* logits_in, float* logits_out, float* thresh_out,
+                        void* ws, cudaStream_t s, bool two_digits = false) {
+    const WsLayout L = workspace_layout(g);
+    uint32_t* err = ws_at<uint32_t>(ws, L.err);
+    const long long rows = static_cast<long long>(g.b) * g.hq;
+    int st;
+    const float* logits = logits_in;
+    if (!logits) {
+        float* dst = logits_out ? logits_out : ws_at<float>(ws, L.logits);
+        if ((st = run_logits(g, dev, q, k, dst, err, s))) return st;
+        logits = dst;
+    }
+    if (N >= g.l) {
+        g_launches += 1;
+        return cuda_status(launch_fill(thresh_out, rows, -std::numeric_limits<float>::infinity(), s));
+    }
+    // tickets (a safety net: they are kept at zero between launches),
+    // histograms and radix state
+    cudaError_t e = cudaMemsetAsync(ws_at<uint8_t>(ws, L.tickets), 0, L.cnt - L.tickets, s);
+    if (e != cudaSuccess) return SAGA_ERR_CUDA;
+    RadixArgs r{};
+    r.passes = two_digits ? kRadixPasses - 1 : kRadixPasses;
+    r.logits = logits;
+    r.rows = rows;
+    r.l = g.l;
+    r.N = N;
+    r.chunks = radix_chunks(rows, g.l, dev.sms);
+    r.hist = ws_at<uint32_t>(ws, L.hist);
+    r.state = ws_at<uint32_t>(ws, L.state);
+    r.tickets = ws_at<uint32_t>(ws, L.tickets);
+    r.thresh = thresh_out;
+    r.err = err;
+    // pass 1 copies every logit at or above its bucket's lower edge out, so
+    // that pass 2 and the compaction of the refresh step read only those
+    r.cand = ws_at<int2>(ws, L.cand);
+    r.cand_cnt = ws_at<int32_t>(ws, L.cand_cnt);
+    g_launches += r.passes;
+    return cuda_status(launch_radix_select(r, s));
+}
+
+// Softmax and gathered value rows over contiguous kept lists (idx, s, cnt,
+// rowmax per row), the last CTA of each row merging its parts into out (or
+// into part's records).
+static int gather_contiguous(const Geometry& g, const DeviceInfo& dev, const void* q, const void* k,
+                             const void* v, const int32_t* idx, const float* sv, const int32_t* cnt,
+                             const float* rowmax, float* out, float* part, int32_t* sel_cnt, void* ws,
+                             const WsLayout& L, cudaStream_t s) {
+    float* records = ws_at<float>(ws, L.records);
+    GatherArgs ga{};
+    ga.g = g;
+    ga.mode = kListContiguous;
+    ga.parts = gather_parts(g, dev);
+    ga.part_major = ga.parts >= kPartMajorParts;
+    ga.max_lists = 1;
+    ga.v = v;
+    ga.idx = idx;
+    ga.list_s = sv;
+    ga.cnt = cnt;
+    ga.rowmax = rowmax;
+    ga.records = records;
+    ga.tickets = ws_at<uint32_t>(ws, L.tickets);
+    ga.err = ws_at<uint32_t>(ws, L.err);
+    ga.cmb.g = g;
+    ga.cmb.mode = kCombineParts;
+    ga.cmb.parts = ga.parts;
+    ga.cmb.records = records;
+    ga.cmb.out = out;
+    ga.cmb.part = part;
+    ga.cmb.sel_cnt = sel_cnt;
+    ga.cmb.empty_rows = part ? nullptr : ws_empty_rows(ws, L);
+    if (part) {  // a shard that kept nothing reports its maxima (recomputed from q and k)
+        ga.cmb.fallback = 1;
+        ga.cmb.q = q;
+        ga.cmb.k = k;
+        ga.cmb.v = v;
+    }
+    g_launches += 1;
+    return cuda_status(launch_gather_pv(ga, s));
+}
+
 extern "C" {
 
 size_t saga_workspace_bytes(const saga_dims* dims, int32_t N) {
-    Geometry g;
+    Geometry g, gd;
+    int k_group = 1;
     if (N <= 0 || make_geometry(dims, &g) != SAGA_OK) return 0;
-    return workspace_layout(g).total;
+    const size_t total = workspace_layout(g).total;
+    // the dense kernel's geometry may hold its partial records differently
+    if (dense_geometry(dims, &gd, &k_group) != SAGA_OK) return total;
+    const size_t dense_total = workspace_layout(gd).total;
+    return dense_total > total ? dense_total : total;
 }
 
 int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const void* k,
@@ -340,41 +455,7 @@ int saga_topn_refresh(const saga_dims* dims, int32_t N, const void* q, const voi
     DeviceInfo dev;
     if ((st = device_info(&dev))) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const WsLayout L = workspace_layout(g);
-    uint32_t* err = ws_at<uint32_t>(ws, L.err);
-    const long long rows = static_cast<long long>(g.b) * g.hq;
-
-    const float* logits = logits_in;
-    if (!logits) {
-        float* dst = logits_out ? logits_out : ws_at<float>(ws, L.logits);
-        if ((st = run_logits(g, dev, q, k, dst, err, s))) return st;
-        logits = dst;
-    }
-    if (N >= g.l) {
-        g_launches += 1;
-        return cuda_status(launch_fill(thresh_out, rows, -std::numeric_limits<float>::infinity(), s));
-    }
-    // tickets (a safety net: they are kept at zero between launches),
-    // histograms and radix state
-    cudaError_t e = cudaMemsetAsync(ws_at<uint8_t>(ws, L.tickets), 0, L.cnt - L.tickets, s);
-    if (e != cudaSuccess) return SAGA_ERR_CUDA;
-    RadixArgs r{};
-    r.logits = logits;
-    r.rows = rows;
-    r.l = g.l;
-    r.N = N;
-    r.chunks = radix_chunks(rows, g.l, dev.sms);
-    r.hist = ws_at<uint32_t>(ws, L.hist);
-    r.state = ws_at<uint32_t>(ws, L.state);
-    r.tickets = ws_at<uint32_t>(ws, L.tickets);
-    r.thresh = thresh_out;
-    r.err = err;
-    // pass 1 copies its bucket's logits into the kept-list region (unused
-    // until the decode call) so that pass 2 reads only those
-    r.cand = ws_at<float>(ws, L.list_idx);
-    r.cand_cnt = ws_at<int32_t>(ws, L.cand_cnt);
-    g_launches += kRadixPasses;
-    return cuda_status(launch_radix_select(r, s));
+    return refresh_impl(g, dev, N, q, k, logits_in, logits_out, thresh_out, ws, s);
 }
 
 // Many records per row (few rows, many slots): several CTAs per row merge
@@ -437,40 +518,16 @@ static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k
         // a shard keeps nothing when nothing passes: the whole row's maxima
         // are found when the shards' records are merged
         sa.keep_max = part ? 0 : 1;
+        sa.empty_rows = part ? nullptr : ws_empty_rows(ws, L);
+        sa.err = err;
         // up to two CTAs per SM of the wide form (its registers) in one wave
         sa.wide = rows <= kSelectWideRowsPerSm * dev.sms;
         cudaError_t e = launch_select_compact(sa, s);
         g_launches += 1;
         if (e != cudaSuccess) return SAGA_ERR_CUDA;
 
-        GatherArgs ga{};
-        ga.g = g;
-        ga.mode = kListContiguous;
-        ga.parts = gather_parts(g, dev);
-        ga.part_major = ga.parts >= kPartMajorParts;
-        ga.max_lists = 1;
-        ga.v = v;
-        ga.idx = sa.idx;
-        ga.list_s = sa.s;
-        ga.cnt = sa.cnt;
-        ga.rowmax = sa.rowmax;
-        ga.records = records;
-        ga.tickets = ws_at<uint32_t>(ws, L.tickets);
-        ga.cmb.g = g;
-        ga.cmb.mode = kCombineParts;
-        ga.cmb.parts = ga.parts;
-        ga.cmb.records = records;
-        ga.cmb.out = out;
-        ga.cmb.part = part;
-        ga.cmb.sel_cnt = sel_cnt;
-        if (part) {  // a shard that kept nothing reports its maxima (recomputed from q and k)
-            ga.cmb.fallback = 1;
-            ga.cmb.q = q;
-            ga.cmb.k = k;
-            ga.cmb.v = v;
-        }
-        g_launches += 1;
-        return cuda_status(launch_gather_pv(ga, s));
+        return gather_contiguous(g, dev, q, k, v, sa.idx, sa.s, sa.cnt, sa.rowmax, out, part, sel_cnt,
+                                 ws, L, s);
     }
 
     // fused: stream K, compare on chip, lists -> gathered PV with the row merge
@@ -509,6 +566,7 @@ static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k
     ga.seg_mall = a.seg_mall;
     ga.records = records;
     ga.tickets = ws_at<uint32_t>(ws, L.tickets);
+    ga.err = err;
     ga.cmb.g = g;
     ga.cmb.mode = kCombineParts;
     ga.cmb.parts = ga.parts;
@@ -521,6 +579,7 @@ static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k
     ga.cmb.part = part;
     ga.cmb.sel_cnt = sel_cnt;
     ga.cmb.sel_idx = sel_idx;
+    ga.cmb.empty_rows = part ? nullptr : ws_empty_rows(ws, L);
     g_launches += 1;
     if ((e = launch_gather_pv(ga, s)) != cudaSuccess || !sel_idx) return cuda_status(e);
 
@@ -533,6 +592,7 @@ static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k
     ia.seg_cnt = a.seg_cnt;
     ia.bitmap = ws_at<uint32_t>(ws, L.logits);
     ia.idx = sel_idx;
+    ia.err = err;
     g_launches += 1;
     return cuda_status(launch_lists_to_index(ia, s));
 }
@@ -543,6 +603,57 @@ int saga_atopn_decode(const saga_dims* dims, const void* q, const void* k, const
     if (!out) return SAGA_ERR_INVALID_ARG;
     return atopn_decode_impl(dims, q, k, v, thresh, logits_in, out, nullptr, sel_idx, sel_cnt, ws,
                              ws_bytes, stream);
+}
+
+int saga_atopn_refresh_step(const saga_dims* dims, int32_t N, const void* q, const void* k,
+                            const void* v, float* thresh_out, float* out, int32_t* sel_idx,
+                            int32_t* sel_cnt, void* ws, size_t ws_bytes, saga_stream_t stream) {
+    Geometry g;
+    int st = make_geometry(dims, &g);
+    if (st) return st;
+    if (N <= 0 || !q || !k || !v || !thresh_out || !out || !aligned(q, 16) || !aligned(k, 16) ||
+        !aligned(v, 16) || !aligned(thresh_out, 4) || !aligned(out, 4))
+        return SAGA_ERR_INVALID_ARG;
+    if ((sel_idx && !aligned(sel_idx, 4)) || (sel_cnt && !aligned(sel_cnt, 4))) return SAGA_ERR_INVALID_ARG;
+    if ((st = check_ws(g, ws, ws_bytes))) return st;
+    DeviceInfo dev;
+    if ((st = device_info(&dev))) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsLayout L = workspace_layout(g);
+    const long long rows = static_cast<long long>(g.b) * g.hq;
+    // few long rows: one compaction CTA per row leaves most SMs idle, and
+    // streaming K again through the fused kernel (the same logits bit for
+    // bit) is faster
+    const bool few_long_rows = rows <= kFusedFewRows && g.l >= kFusedMinPositions;
+    // every entry kept, or a row whose bitmap does not fit on chip: the
+    // compaction reads the stored logits
+    const bool from_candidates = N < g.l && !few_long_rows &&
+                                 cand_select_smem(g.l) <= static_cast<size_t>(dev.max_smem);
+    if ((st = refresh_impl(g, dev, N, q, k, nullptr, nullptr, thresh_out, ws, s, from_candidates)))
+        return st;
+    if (!from_candidates) {
+        const float* logits_in = few_long_rows && N < g.l ? nullptr : ws_at<float>(ws, L.logits);
+        return atopn_decode_impl(dims, q, k, v, thresh_out, logits_in, out, nullptr, sel_idx, sel_cnt, ws,
+                                 ws_bytes, stream);
+    }
+    CandSelectArgs ca{};
+    ca.cand = ws_at<int2>(ws, L.cand);
+    ca.cand_cnt = ws_at<int32_t>(ws, L.cand_cnt);
+    ca.chunks = radix_chunks(rows, g.l, dev.sms);  // as the radix passes cut the rows
+    ca.state = ws_at<uint32_t>(ws, L.state);       // the last digit is found here
+    ca.thresh = thresh_out;
+    ca.rows = rows;
+    ca.l = g.l;
+    ca.idx = sel_idx ? sel_idx : ws_at<int32_t>(ws, L.list_idx);
+    ca.s = ws_at<float>(ws, L.list_s);
+    ca.cnt = ws_at<int32_t>(ws, L.cnt);
+    ca.rowmax = ws_at<float>(ws, L.rowmax);
+    ca.empty_rows = ws_empty_rows(ws, L);
+    ca.err = ws_at<uint32_t>(ws, L.err);
+    g_launches += 1;
+    if (launch_cand_select(ca, s) != cudaSuccess) return SAGA_ERR_CUDA;
+    return gather_contiguous(g, dev, q, k, v, ca.idx, ca.s, ca.cnt, ca.rowmax, out, nullptr, sel_cnt, ws,
+                             L, s);
 }
 
 int saga_atopn_decode_partial(const saga_dims* dims, const void* q, const void* k, const void* v,
@@ -634,7 +745,8 @@ int saga_topn_select_digit(const saga_dims* dims, int32_t N, int32_t pass, const
 int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const void* v,
                       float* out, void* ws, size_t ws_bytes, saga_stream_t stream) {
     Geometry g;
-    int st = make_geometry(dims, &g);
+    int k_group = 1;
+    int st = dense_geometry(dims, &g, &k_group);
     if (st) return st;
     if (!dense_supported(g)) return SAGA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !out || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
@@ -651,10 +763,11 @@ int saga_decode_dense(const saga_dims* dims, const void* q, const void* k, const
     if (dense_smem_bytes(g, stages) > static_cast<size_t>(dev.max_smem)) return SAGA_ERR_UNSUPPORTED;
 
     CUtensorMap kmap, vmap;
-    if ((st = encode_cache_map(&kmap, k, g, g.hk, g.d))) return st;
+    if ((st = encode_cache_map(&kmap, k, g, g.hk / k_group, g.d))) return st;
     if ((st = encode_cache_map(&vmap, v, g, g.hv, g.dv))) return st;
     DenseArgs a{};
     a.g = g;
+    a.k_group = k_group;
     a.C = stream_ctas(g, dev, 1);
     a.stages = stages;
     a.q = q;
@@ -718,7 +831,21 @@ int saga_workspace_error(void* ws, size_t ws_bytes, saga_stream_t stream) {
     if (cudaMemcpy(&word, ws, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
         return SAGA_ERR_CUDA;
     if (word && cudaMemset(ws, 0, sizeof word) != cudaSuccess) return SAGA_ERR_CUDA;
-    return (word & kErrTimeout) ? SAGA_ERR_TIMEOUT : SAGA_OK;
+    if (word & kErrTimeout) return SAGA_ERR_TIMEOUT;
+    return (word & kErrBounds) ? SAGA_ERR_BOUNDS : SAGA_OK;
+}
+
+int saga_workspace_empty_rows(void* ws, size_t ws_bytes, uint64_t* count_out, saga_stream_t stream) {
+    if (!ws || ws_bytes < 256 || !count_out) return SAGA_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    uint32_t* counter = reinterpret_cast<uint32_t*>(ws) + 1;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SAGA_ERR_CUDA;
+    if (cudaMemcpy(&word, counter, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SAGA_ERR_CUDA;
+    if (word && cudaMemset(counter, 0, sizeof word) != cudaSuccess) return SAGA_ERR_CUDA;
+    *count_out = word;
+    return SAGA_OK;
 }
 
 const char* saga_status_string(int status) {
@@ -730,6 +857,7 @@ const char* saga_status_string(int status) {
         case SAGA_ERR_CUDA: return "CUDA error";
         case SAGA_ERR_DEVICE: return "no sm_100 device";
         case SAGA_ERR_TIMEOUT: return "a bounded device wait timed out";
+        case SAGA_ERR_BOUNDS: return "an index out of range (debug build check)";
         default: return "unknown status";
     }
 }

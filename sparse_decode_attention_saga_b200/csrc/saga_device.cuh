@@ -46,6 +46,22 @@ __device__ __forceinline__ void raise_device_error(uint32_t* err_word, uint32_t 
     if (err_word) atomicOr(err_word, bit);
 }
 
+// Debug builds (-DSAGA_DEBUG) check every position, count and slot a kernel
+// takes from another kernel's output before it uses it: a value out of range
+// sets kErrBounds in the sticky flag and the caller skips the access (no
+// trap: the context stays usable and saga_workspace_error reports it).
+// Release builds compile the checks away (always in bounds).
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t* err_word) {
+#ifdef SAGA_DEBUG
+    if (!ok) raise_device_error(err_word, kErrBounds);
+    return ok;
+#else
+    (void)ok;
+    (void)err_word;
+    return true;
+#endif
+}
+
 // ----------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

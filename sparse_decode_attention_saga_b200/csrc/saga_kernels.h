@@ -30,10 +30,12 @@ cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-// Raises the dynamic shared-memory limit of kernel `fn` to `bytes` on the
-// current device.  CUDA keeps function attributes per device, so this is
-// done once per (kernel, device) and remembered (a process that drives
-// several GPUs sets it on each before the kernel's first launch there).
+// Makes kernel `fn` launchable with `bytes` of dynamic shared memory on the
+// current device: above the 48 KB default the limit is raised, to the
+// largest value asked for so far (never lowered).  CUDA keeps function
+// attributes per device, so the limit is remembered per (kernel, device) (a
+// process that drives several GPUs sets it on each before the kernel's
+// first launch there).
 cudaError_t allow_dynamic_smem(const void* fn, int bytes);
 template <typename... KArgs>
 cudaError_t allow_dynamic_smem(void (*kern)(KArgs...), int bytes) {
@@ -75,16 +77,23 @@ struct RadixArgs {
     uint32_t* tickets;
     float* thresh;
     uint32_t* err;
-    // Optional (nullable): pass 1 also copies the logits of its prefix bucket
-    // into chunk c's part [c*per, c*per + per) of cand[row][0..l) and their
-    // number into cand_cnt[row][c]; pass 2 then reads only those (chunk c's
-    // CTA its own chunk's).  Null: pass 2 reads the whole row again.
-    float* cand;
+    // Digits to find (3: the whole threshold; 2: stop after pass 1 and leave
+    // the last digit to the candidate compaction, which reads `state`).
+    int passes;
+    // Optional (nullable): pass 1 also copies (position, logit bits) of every
+    // logit whose key is at or above the lower edge of pass 0's bucket into
+    // chunk c's part [c*per, c*per + per) of cand[row][0..l) (per =
+    // radix_chunk_len, in no fixed order) and their number into
+    // cand_cnt[row][c]; pass 2 then reads only those (chunk c's CTA its own
+    // chunk's).  Null: pass 2 reads the whole row again.
+    int2* cand;
     int32_t* cand_cnt;
 };
 cudaError_t launch_radix_select(const RadixArgs& a, cudaStream_t stream);
 // CTAs per row for the radix passes (cost model over waves and per-CTA overhead).
 int radix_chunks(long long rows, int l, int sms);
+// Positions per chunk of a row cut into `chunks` (a multiple of 4).
+SAGA_HD int radix_chunk_len(int l, int chunks) { return ((l + chunks - 1) / chunks + 3) & ~3; }
 // Adds n to the library's launch counter (saga_launch_count).
 void note_launches(int n);
 cudaError_t launch_fill(float* p, long long n, float value, cudaStream_t stream);
@@ -101,8 +110,35 @@ struct SelectArgs {
     float* rowmax; // [rows]     largest logit of the row
     int keep_max;  // nothing passed: keep the row's maxima (1) or nothing (0)
     int wide;      // few rows: 16 logits per thread per sub-round instead of 4
+    uint32_t* empty_rows;  // optional: counts the rows that kept their maxima
+    uint32_t* err;         // sticky flag (debug builds: bounds checks)
 };
 cudaError_t launch_select_compact(const SelectArgs& a, cudaStream_t stream);
+
+// The same compare and ordered compaction over the candidates of the radix
+// passes (RadixArgs::cand: every logit at or above the lower edge of the
+// threshold's first-digit bucket, so every kept one, and the row's largest),
+// one CTA per row with the row's bitmap of kept positions in shared memory.
+// With `state` (the radix state after the first two digits), the kernel
+// also finds the threshold's last digit from the candidates and writes the
+// thresholds (the radix passes then stop after two digits).
+struct CandSelectArgs {
+    const int2* cand;          // [rows][l]  (position, logit bits), chunk c at c*per
+    const int32_t* cand_cnt;   // [rows][kRadixMaxChunks]
+    int chunks;                // the radix passes' chunks per row
+    const uint32_t* state;     // nullable [rows][2]: (22-bit prefix, rank) after two digits
+    float* thresh;             // [rows]: in, or out with state
+    long long rows;
+    int l;
+    int32_t* idx;   // [rows][l]  kept positions, ascending
+    float* s;       // [rows][l]  their logits, same order
+    int32_t* cnt;   // [rows]
+    float* rowmax;  // [rows]     largest logit of the row
+    uint32_t* empty_rows;  // optional: counts the rows that kept their maxima
+    uint32_t* err;         // sticky flag (debug builds: bounds checks)
+};
+size_t cand_select_smem(int l);
+cudaError_t launch_cand_select(const CandSelectArgs& a, cudaStream_t stream);
 
 // Ascending kept positions of every row from the fused kernel's per-(slot,
 // warp) lists: the lists' positions are set in a per-row bitmap, which is
@@ -115,6 +151,7 @@ struct IndexArgs {
     const int32_t* seg_cnt;  // [rows][S_cap][WPK]
     uint32_t* bitmap;        // scratch [rows][ceil(l/32)]
     int32_t* idx;            // [rows][l] out
+    uint32_t* err;           // sticky flag (debug builds: bounds checks)
 };
 cudaError_t launch_lists_to_index(const IndexArgs& a, cudaStream_t stream);
 
@@ -147,6 +184,9 @@ struct CombineArgs {
     // (count 0: m = -inf, l = number of positions at the row max, o = the
     // sum of their value rows).
     float* part;
+    // Optional: counts the rows that kept nothing and took the empty-set
+    // fallback (one atomic add per such row; not for a shard's partials).
+    uint32_t* empty_rows;
 };
 // Gathered softmax-PV over kept lists -> partial records.
 enum ListMode : int {
@@ -173,6 +213,7 @@ struct GatherArgs {
     // zero) merges the row's `parts` records as cmb describes.
     uint32_t* tickets;
     CombineArgs cmb;
+    uint32_t* err;  // sticky flag (debug builds: bounds checks)
 };
 size_t gather_smem_bytes(int max_lists);
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream);
@@ -182,12 +223,18 @@ struct DenseArgs {
     Geometry g;
     int C;
     int stages;
+    // Key heads of g per key head of the cache (1, or h_v / h_k when more
+    // than two value heads share a key head: g then has one key head per
+    // value head, and key head kh of g loads the cache's key head
+    // kh / k_group, so that each such head's query heads use one value head).
+    int k_group;
     const void* q;
     float* records;
     uint32_t* err;
 };
 // Shapes the dense kernel handles: h_v <= 2 h_k, value heads aligned with
-// the key-head groups.
+// the key-head groups (geometries with more value heads per key head go
+// through the k_group form above).
 bool dense_supported(const Geometry& g);
 size_t dense_stage_bytes(const Geometry& g);
 size_t dense_smem_bytes(const Geometry& g, int stages);

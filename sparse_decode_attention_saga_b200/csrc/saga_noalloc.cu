@@ -99,6 +99,7 @@ extern "C" int saga_topn_refresh_noalloc(const saga_dims* dims, int32_t N, const
     if (cudaMemsetAsync(scratch, 0, static_cast<size_t>(rows) * kRowBytes, s) != cudaSuccess)
         return SAGA_ERR_CUDA;
     RadixArgs r{};
+    r.passes = kRadixPasses;
     r.logits = logits_in;
     r.rows = rows;
     r.l = l;

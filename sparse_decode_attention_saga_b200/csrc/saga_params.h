@@ -29,6 +29,9 @@ constexpr int kGatherMaxSmem = 96 * 1024;
 // Bounded device waits give up after this long and raise kErrTimeout.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 constexpr uint32_t kErrTimeout = 1u;
+// Debug builds (SAGA_DEBUG): an index read from another kernel's output was
+// out of range (the access was skipped).
+constexpr uint32_t kErrBounds = 2u;
 // Radix select: 32-bit keys in digits of 11, 11 and 10 bits.
 constexpr int kRadixBins = 2048;
 constexpr int kRadixPasses = 3;
@@ -88,7 +91,7 @@ SAGA_HD SegList seg_list_of(int P, int MBW, int WPK, int tiles, int bb, int j, l
 // growing cache); the per-row tickets, which must be zero on entry, live
 // there.
 struct WsLayout {
-    size_t err;       // uint32 sticky flag (256-byte header)
+    size_t err;       // uint32 sticky flag, then the uint32 empty-set row counter (256-byte header)
     size_t tickets;   // uint32 [b*hq]  last-CTA tickets (zero on entry, left at zero)
     size_t hist;      // uint32 [kRadixPasses][b*hq][kRadixBins]
     size_t state;     // uint32 [b*hq][2]  (prefix, rank)
@@ -101,6 +104,7 @@ struct WsLayout {
     size_t list_idx;  // int32  [b*hq][l_pad]; with list_s also the int2 [b*hq][l_pad]
     size_t list_s;    // float  [b*hq][l_pad]   (position, logit) pairs of the fused path
     size_t logits;    // float  [b*hq][l]
+    size_t cand;      // int2   [b*hq][l]  radix pass-1 candidates (position, logit bits)
     size_t total;
 };
 
@@ -128,6 +132,7 @@ inline WsLayout workspace_layout(const Geometry& g) {
     w.list_idx = take(rows * g.l_pad * sizeof(int32_t));
     w.list_s = take(rows * g.l_pad * sizeof(float));
     w.logits = take(rows * g.l * sizeof(float));
+    w.cand = take(rows * g.l * 2 * sizeof(int32_t));
     w.total = off;
     return w;
 }

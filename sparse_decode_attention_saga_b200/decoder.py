@@ -6,7 +6,7 @@ refresh schedule of "More Value per Key" (ai.info summary, Key Contributions
 #2: the exact threshold is recomputed on every n-th token only and reused on
 the tokens in between):
 step t refreshes when t mod n == 0, then decodes with the stored thresholds.
-Every step is two or three C calls; all compute runs in libsaga.so.
+Every step is one C call; all compute runs in libsaga.so.
 ``HostLoop`` (``AtopNDecoder.host_loop``) runs a span of steps as one CUDA
 graph fed from, and writing to, pinned host memory.
 """
@@ -66,16 +66,17 @@ class AtopNDecoder:
         return t % self.n == 0
 
     def refresh(self, q, k, stream=None) -> None:
-        """Exact thresholds from this step's logits (kept in self.logits)."""
+        """Exact thresholds from this step's logits (kept in self.logits);
+        ``step`` refreshes through the workspace instead, in the same call as
+        the decode."""
         _lib.topn_refresh(self.dims, self.N, q, k, None, self.logits, self.thresh, self.ws, stream)
 
     def step(self, t: int, q, k, v, out=None, sel_idx=None, sel_cnt=None, stream=None):
         """Decode step t: refresh if t mod n == 0, then Atop-N attention."""
         out = self.out if out is None else out
         if self.is_refresh(t):
-            self.refresh(q, k, stream)
-            _lib.atopn_decode(self.dims, q, k, v, self.thresh, self.logits, out, sel_idx, sel_cnt,
-                              self.ws, stream)
+            _lib.atopn_refresh_step(self.dims, self.N, q, k, v, self.thresh, out, sel_idx, sel_cnt,
+                                    self.ws, stream)
         else:
             _lib.atopn_decode(self.dims, q, k, v, self.thresh, None, out, sel_idx, sel_cnt,
                               self.ws, stream)
@@ -88,6 +89,11 @@ class AtopNDecoder:
 
     def error(self, stream=None) -> int:
         return _lib.workspace_error(self.ws, stream)
+
+    def empty_rows(self, stream=None) -> int:
+        """Rows that kept nothing and took the empty-set rule (their maxima)
+        since the last call."""
+        return _lib.workspace_empty_rows(self.ws, stream)
 
     def host_loop(self, k, v, q_host, out_host, t0: int, steps: int, stream=None,
                   restore: bool = True) -> "HostLoop":

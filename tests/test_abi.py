@@ -41,8 +41,17 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
+def test_debug_library_exports_every_declared_symbol():
+    """The bounds-checked build (SAGA_DEBUG) has the same boundary."""
+    if not os.path.exists(_lib.DEBUG_LIBRARY):
+        saga_build.build(debug=True)
+    dbg = ctypes.CDLL(_lib.DEBUG_LIBRARY)
+    for name in declared_functions():
+        assert hasattr(dbg, name), name
+
+
 def test_status_strings(lib):
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         assert _lib.status_string(code) not in ("", "unknown status")
     assert _lib.status_string(-99) == "unknown status"
 
@@ -93,8 +102,9 @@ def test_pointer_and_workspace_validation(lib):
     # N <= 0
     assert lib.saga_topn_refresh(ctypes.byref(d), 0, 16, 16, None, None, 16, base, need,
                                  None) == _lib.SAGA_ERR_INVALID_ARG
-    # dense needs h_v <= 2 h_k
-    d2 = _lib.dims(1, 8, 1, 8, 64, 64)
+    # dense: more than two value heads per key head only when each value
+    # head can stand as a key head of its own (h_v in {1, 2, 4, 8})
+    d2 = _lib.dims(1, 12, 2, 6, 64, 64)
     n2 = _lib.workspace_bytes(d2, 8)
     ws2 = _ws(n2 + 512)
     b2 = (ws2.data_ptr() + 255) // 256 * 256

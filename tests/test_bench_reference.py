@@ -23,8 +23,12 @@ def test_reference_arm_prints_the_contract_line():
     assert d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
     assert d["value"] > 0 and abs(d["ms_per_step"] * 1e3 - d["value"]) < 1e-6 * d["value"]
     assert d["config"]["workload"] == "tiny"
+    # the same config keys as the GPU arm's line
+    assert set(d["config"]) == {"workload", "batch", "h_q", "h_k", "h_v", "head_dim", "v_head_dim",
+                                "l_kv", "N", "n", "parallelism", "l2", "timing"}
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"]
+    assert cb["cores"] == len(os.sched_getaffinity(0))
     assert cb["sample"].startswith("oracle steps 1..2 ")  # the timed steps follow the warm-up
     e = d["e2e"]
     assert e["value"] == d["value"] and e["h2d_bytes_per_step"] == 0 == e["d2h_bytes_per_step"]

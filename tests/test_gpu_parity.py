@@ -103,8 +103,7 @@ def test_mask_bit_exact_and_output_given_mask(shape):
     qs, K, V = device_inputs(w, seed=4, steps=2)
     dec = AtopNDecoder.for_workload(w)
     out, idx, cnt = gpu_step_with_mask(dec, 0, qs[0], K, V)   # refresh step
-    torch.cuda.synchronize()
-    s = dec.logits.cpu().numpy()
+    s = gpu_logits(dec, qs[0], K).cpu().numpy()
     tau = dec.thresh.cpu().numpy()
     mask_gpu = mask_from_lists(idx, cnt, w.l_kv)
     mask_ref, cnt_ref = oracle.select(s, tau)
@@ -161,18 +160,22 @@ def test_stale_threshold_above_every_logit_keeps_the_maxima(shape):
     torch.cuda.synchronize()
     s = dec.logits.cpu().numpy()
     dec.thresh.copy_(torch.from_numpy(s.max(-1) + 1.0))
+    assert dec.empty_rows() == 0
     # fused path (fallback in the combine kernel)
     out_fused = torch.empty_like(dec.out)
     cnt_fused = torch.zeros((w.batch, w.h_q), dtype=torch.int32, device="cuda")
     idx_fused = torch.full((w.batch, w.h_q, w.l_kv), -1, dtype=torch.int32, device="cuda")
     _lib.atopn_decode(dec.dims, qs[0], K, V, dec.thresh, None, out_fused, idx_fused, cnt_fused,
                       dec.ws)
+    rows = w.batch * w.h_q
+    assert dec.empty_rows() == rows   # every row took the rule, counted once
     # stored-logits path
     out_l, idx, cnt = torch.empty_like(dec.out), None, None
     idx = torch.full((w.batch, w.h_q, w.l_kv), -1, dtype=torch.int32, device="cuda")
     cnt = torch.zeros((w.batch, w.h_q), dtype=torch.int32, device="cuda")
     _lib.atopn_decode(dec.dims, None, None, V, dec.thresh, dec.logits, out_l, idx, cnt, dec.ws)
     torch.cuda.synchronize()
+    assert dec.empty_rows() == rows
     mask_ref, cnt_ref = oracle.select(s, dec.thresh.cpu().numpy())
     assert np.array_equal(mask_from_lists(idx, cnt, w.l_kv), mask_ref)
     assert np.array_equal(cnt_fused.cpu().numpy(), cnt_ref)
@@ -237,7 +240,8 @@ def test_refresh_every_step_is_exact_topN():
 
 # ---------------------------------------------------------------- dense (a7)
 
-@pytest.mark.parametrize("s", [x for x in SHAPES if x[4] <= 2 * x[3]], ids=lambda x: x[0])
+@pytest.mark.parametrize("s", [x for x in SHAPES if x[4] <= 2 * x[3] or x[4] in (4, 8)],
+                         ids=lambda x: x[0])
 def test_dense_matches_oracle(s):
     w = wl(*s)
     qs, K, V = device_inputs(w, seed=8, steps=1)

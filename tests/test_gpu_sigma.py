@@ -39,19 +39,22 @@ def test_sigma_decode_loop_matches_oracle(s):
     run_loop_and_compare(_w(*s), seed=31)
 
 
-def test_sigma_full_attention_matches_oracle_dense():
-    """N >= l keeps everything: full attention, against the oracle's.  (The
-    dense kernel does not take this shape: with four value heads per key head
-    a stage's value rows are 4x its 32 KB of keys.)"""
-    w = _w("sigma_full", 1, 16, 2, 8, 400, None, N=400, steps=1)
+@pytest.mark.parametrize("s", SIGMA, ids=lambda s: s[0])
+def test_sigma_full_attention_matches_oracle_dense(s):
+    """N >= l keeps everything: full attention, against the oracle's, and the
+    dense kernel (four value heads per key head: one key head per value head,
+    each reading its key head's rows) against the same."""
+    name, b, hq, hk, hv, l, _ = s
+    w = _w(name, b, hq, hk, hv, min(l, 400), None, N=400, steps=1)
     qs, K, V = device_inputs(w, seed=33, steps=1)
     dec = AtopNDecoder.for_workload(w)
     out_a = dec.step(0, qs[0], K, V).clone()
+    out_d = dec.dense(qs[0], K, V).clone()
     torch.cuda.synchronize()
     ref = oracle.decode_dense(bits(qs[0]), bits(K), bits(V))
     assert_outputs_close(out_a.cpu().numpy(), ref, "N >= l")
-    with pytest.raises(_lib.SagaError):
-        dec.dense(qs[0], K, V)
+    assert_outputs_close(out_d.cpu().numpy(), ref, "dense")
+    assert dec.error() == _lib.SAGA_OK
 
 
 def test_narrow_keys_dense_where_it_fits():
