@@ -19,8 +19,10 @@
 // row and no row waits for a second wave of CTAs that turn out to be empty.
 // Each warp then works through its own contiguous part of that share without
 // block barriers: 32 entries at a time, one (position, logit) per lane read
-// with coalesced loads one round ahead, and 16-byte value-row loads by lane
-// groups (8 or 16 lanes per row), weighted by exp(s - m) and accumulated in
+// with coalesced loads, the 32 value rows copied with cp.async into a
+// two-stage per-warp ring in shared memory (the next 32 rows' loads in
+// flight while these are summed), and each row read back by a lane group
+// (8 or 16 lanes, 16 bytes each), weighted by exp(s - m) and accumulated in
 // fp32.  m is the row's largest logit, which is always kept when anything is
 // (tau_eff <= max), so no running max is needed.  The share's (m, sum of
 // weights, count, row max, unnormalised output) record is merged across
@@ -35,24 +37,41 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMinShare = 128;  // kept entries per CTA at least
-#ifndef SAGA_GATHER_INFLIGHT
-#define SAGA_GATHER_INFLIGHT 2
+#ifndef SAGA_GATHER_STAGES
+#define SAGA_GATHER_STAGES 2
 #endif
 #ifndef SAGA_GATHER_MINBLOCKS
-#define SAGA_GATHER_MINBLOCKS 4
+#define SAGA_GATHER_MINBLOCKS 3
 #endif
-// value-row loads in flight per lane group, and CTAs per SM the register
-// budget is sized for (tuning constants)
-constexpr int kGatherInflight = SAGA_GATHER_INFLIGHT;
-constexpr int kGatherMinBlocks = SAGA_GATHER_MINBLOCKS;
+// CTAs per SM the register budget is sized for with the stage ring (a
+// tuning constant; its shared memory allows three with two stages), four
+// without
+template <bool STAGED>
+constexpr int gather_min_blocks() { return STAGED ? SAGA_GATHER_MINBLOCKS : 4; }
 
 static_assert(kThreads == kCombineThreads, "the last CTA of a row runs the row merge");
 
+// Per-warp ring of value-row stages (cp.async, 64-dim value heads): 32 rows
+// of the value head dim, then the 32 entries' weights.  128-dim value heads
+// load their rows into registers, kGatherInflight per lane at a time.
+constexpr int kGatherStages = SAGA_GATHER_STAGES;
+constexpr int kGatherInflight = 2;
+template <int D>
+struct GatherStage {
+    static constexpr int kRowsBytes = 32 * D * 2;
+    static constexpr int kBytes = kRowsBytes + 32 * 4;
+};
+__host__ __device__ inline size_t gather_ring_offset(int max_lists) {
+    return ((2 * static_cast<size_t>(max_lists) + 1) * sizeof(int) + 127) / 128 * 128;
+}
+
 // D: value head dim, DK: key/query head dim, PM: part-major grid (rows, parts)
-template <int D, int DK, int NT, bool PM>
-__global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(const GatherArgs a) {
+// STAGED: the value rows go through the cp.async ring (64-dim value heads).
+template <int D, int DK, int NT, bool PM, bool STAGED>
+__global__ void __launch_bounds__(kThreads, gather_min_blocks<STAGED>()) gather_pv_kernel(const GatherArgs a) {
     constexpr int LPR = D * 2 / 16;    // lanes per value row (16 B each)
     constexpr int RPI = 32 / LPR;      // value rows per warp instruction
+    constexpr bool kStaged = STAGED && D == 64;  // value rows through the cp.async ring
 
     extern __shared__ int table[];     // pre, start
     __shared__ float red_m[kWarps];
@@ -187,11 +206,10 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] = 0.f;
     float lsum = 0.f;
-    const __nv_bfloat16* vbase = reinterpret_cast<const __nv_bfloat16*>(a.v) +
-                                 (static_cast<size_t>(bb) * g.l_cap * g.hv + vh) * D + col0;
-    const size_t vstride = static_cast<size_t>(g.hv) * D;
-    constexpr int ROUNDS = 32 / RPI;   // value-row loads per lane per 32 entries
-    constexpr int INFLIGHT = ROUNDS < kGatherInflight ? ROUNDS : kGatherInflight;
+    const char* vrow0 = reinterpret_cast<const char*>(a.v) +
+                        (static_cast<size_t>(bb) * g.l_cap * g.hv + vh) * D * 2;
+    const size_t vstride = static_cast<size_t>(g.hv) * D * 2;  // bytes between positions
+    constexpr int ROUNDS = 32 / RPI;   // value rows per lane group per 32 entries
 
     // entry e -> (position, logit); out-of-range entries give (0, -inf)
     // The list holding entry e is the last j with pre[j] <= e.  Each lane's
@@ -229,38 +247,110 @@ __global__ void __launch_bounds__(kThreads, kGatherMinBlocks) gather_pv_kernel(c
             }
         }
     };
-    int nxt_pos;
-    float nxt_s;
-    fetch(w0 + lane, nxt_pos, nxt_s);
-    for (int base = w0; base < w1; base += 32) {
-        // one entry per lane; the next round's entries are already in flight
-        const int pos = nxt_pos;
-        const float s = nxt_s;
-        fetch(base + 32 + lane, nxt_pos, nxt_s);
-        const float p_lane = base + lane < w1 ? __expf(s - m) : 0.f;
-        lsum += p_lane;
-        // lane group grp gathers entries grp, grp+RPI, ... of the 32
+
+    const int grp_col = (lane % LPR) * 16;  // this lane's 16 bytes of a value row
+    if constexpr (kStaged) {
+        // Value rows of 32 entries at a time go to a per-warp ring of
+        // kGatherStages stages in shared memory with cp.async (16 bytes per
+        // lane and copy, zeros for entries past the share), so that the
+        // loads of the next stage are in flight while this one is summed;
+        // each stage also holds its entries' weights exp(s - m).  The
+        // entries of the next stage to issue are fetched one issue ahead.
+        uint8_t* ring = reinterpret_cast<uint8_t*>(table) + gather_ring_offset(a.max_lists) +
+                        static_cast<size_t>(warp) * kGatherStages * GatherStage<D>::kBytes;
+        int nxt_pos;
+        float nxt_s;
+        fetch(w0 + lane, nxt_pos, nxt_s);
+        auto issue = [&](int st, int e_base) {
+            const int pos = nxt_pos;
+            const float s = nxt_s;
+            uint8_t* rows = ring + st * GatherStage<D>::kBytes;
+            reinterpret_cast<float*>(rows + GatherStage<D>::kRowsBytes)[lane] =
+                e_base + lane < w1 ? __expf(s - m) : 0.f;
+            const uint32_t rows_a = smem_addr(rows);
 #pragma unroll
-        for (int r0 = 0; r0 < ROUNDS; r0 += INFLIGHT) {
-            uint4 raw[INFLIGHT];
-#pragma unroll
-            for (int u = 0; u < INFLIGHT; ++u) {
-                const int k = (r0 + u) * RPI + grp;
-                const int pk = __shfl_sync(0xffffffffu, pos, k);
-                raw[u] = base + k < w1 ? __ldg(reinterpret_cast<const uint4*>(vbase + pk * vstride))
-                                       : make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < LPR; ++i) {
+                const int q = i * 32 + lane;  // 16-byte chunk q: row q / LPR, column chunk q % LPR
+                const int r = q / LPR, cc = q % LPR;
+                const int pr = __shfl_sync(0xffffffffu, pos, r);
+                cp_async_16(rows_a + r * (D * 2) + cc * 16, vrow0 + static_cast<size_t>(pr) * vstride + cc * 16,
+                            e_base + r < w1 ? 16u : 0u);
             }
-            float p[INFLIGHT];
+            cp_async_commit();
+            fetch(e_base + 32 + lane, nxt_pos, nxt_s);
+        };
+        auto consume = [&](int st) {
+            const uint8_t* rows = ring + st * GatherStage<D>::kBytes;
+            const float* pw = reinterpret_cast<const float*>(rows + GatherStage<D>::kRowsBytes);
+            lsum += pw[lane];
 #pragma unroll
-            for (int u = 0; u < INFLIGHT; ++u)
-                p[u] = __shfl_sync(0xffffffffu, p_lane, (r0 + u) * RPI + grp);
-#pragma unroll
-            for (int u = 0; u < INFLIGHT; ++u) {
-                const uint32_t w4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+            for (int r0 = 0; r0 < ROUNDS; ++r0) {
+                const int r = r0 * RPI + grp;
+                const uint4 raw = *reinterpret_cast<const uint4*>(rows + r * (D * 2) + grp_col);
+                const float p = pw[r];
+                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    acc[2 * c] = fmaf(p[u], bf16_lo(w4[c]), acc[2 * c]);
-                    acc[2 * c + 1] = fmaf(p[u], bf16_hi(w4[c]), acc[2 * c + 1]);
+                    acc[2 * c] = fmaf(p, bf16_lo(w4[c]), acc[2 * c]);
+                    acc[2 * c + 1] = fmaf(p, bf16_hi(w4[c]), acc[2 * c + 1]);
+                }
+            }
+        };
+        const int nr = (w1 - w0 + 31) / 32;  // rounds of this warp
+#pragma unroll
+        for (int st = 0; st < kGatherStages; ++st) {
+            if (st < nr) issue(st, w0 + st * 32);
+            else cp_async_commit();  // empty groups keep the count of pending groups uniform
+        }
+        for (int it = 0; it < nr; ++it) {
+            const int st = it % kGatherStages;
+            cp_async_wait<kGatherStages - 1>();  // this lane's copies of round it are done
+            __syncwarp();                        // and every lane's
+            consume(st);
+            __syncwarp();                        // the stage is free again
+            if (it + kGatherStages < nr) issue(st, w0 + (it + kGatherStages) * 32);
+            else cp_async_commit();
+        }
+        cp_async_wait<0>();
+    } else {
+        // Few entries per warp, or 128-dim value rows (the ring would leave
+        // one CTA per SM): the rows are loaded into registers,
+        // kGatherInflight per lane at a time, with the next round's entries
+        // in flight.
+        int nxt_pos;
+        float nxt_s;
+        fetch(w0 + lane, nxt_pos, nxt_s);
+        constexpr int INFLIGHT = ROUNDS < kGatherInflight ? ROUNDS : kGatherInflight;
+        for (int base = w0; base < w1; base += 32) {
+            const int pos = nxt_pos;
+            const float s = nxt_s;
+            fetch(base + 32 + lane, nxt_pos, nxt_s);
+            const float p_lane = base + lane < w1 ? __expf(s - m) : 0.f;
+            lsum += p_lane;
+            // lane group grp gathers entries grp, grp+RPI, ... of the 32
+#pragma unroll
+            for (int r0 = 0; r0 < ROUNDS; r0 += INFLIGHT) {
+                uint4 raw[INFLIGHT];
+#pragma unroll
+                for (int u = 0; u < INFLIGHT; ++u) {
+                    const int k = (r0 + u) * RPI + grp;
+                    const int pk = __shfl_sync(0xffffffffu, pos, k);
+                    raw[u] = base + k < w1 ? __ldg(reinterpret_cast<const uint4*>(
+                                                 vrow0 + static_cast<size_t>(pk) * vstride + grp_col))
+                                           : make_uint4(0u, 0u, 0u, 0u);
+                }
+                float pu[INFLIGHT];
+#pragma unroll
+                for (int u = 0; u < INFLIGHT; ++u)
+                    pu[u] = __shfl_sync(0xffffffffu, p_lane, (r0 + u) * RPI + grp);
+#pragma unroll
+                for (int u = 0; u < INFLIGHT; ++u) {
+                    const uint32_t w4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        acc[2 * c] = fmaf(pu[u], bf16_lo(w4[c]), acc[2 * c]);
+                        acc[2 * c + 1] = fmaf(pu[u], bf16_hi(w4[c]), acc[2 * c + 1]);
+                    }
                 }
             }
         }
@@ -314,6 +404,20 @@ size_t gather_smem_bytes(int max_lists) {
     return (2 * static_cast<size_t>(max_lists) + 1) * sizeof(int);
 }
 
+static size_t gather_total_smem(int max_lists, bool staged) {
+    if (!staged) return gather_smem_bytes(max_lists);  // no ring
+    return gather_ring_offset(max_lists) + static_cast<size_t>(kWarps) * kGatherStages * GatherStage<64>::kBytes;
+}
+
+// The ring pays where each warp has many rounds of 32 entries (long rows,
+// many of them: Llama-shaped batch 16 at 128K, 44.7 against 52.9 us for the
+// gather with its merge); with few entries per warp its extra latency and
+// the lower occupancy cost more (batch 1 at 128K: 12.3 against 7.1 us;
+// batch 16 at 8K: 26.1 against 22.8 us).
+static bool gather_staged(const Geometry& g) {
+    return g.dv == 64 && g.l >= 65536 && static_cast<long long>(g.b) * g.hq >= 128;
+}
+
 
 cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
     const long long rows = static_cast<long long>(a.g.b) * a.g.hq;
@@ -321,23 +425,29 @@ cudaError_t launch_gather_pv(const GatherArgs& a, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     const dim3 grid = a.part_major ? dim3(static_cast<unsigned>(rows), static_cast<unsigned>(a.parts))
                                    : dim3(static_cast<unsigned>(a.parts), static_cast<unsigned>(rows));
-    const size_t smem = gather_smem_bytes(a.max_lists);
-    if (smem > static_cast<size_t>(kGatherMaxSmem) || a.cmb.parts != a.parts) return cudaErrorInvalidValue;
-#define SAGA_GATHER_CASE(D_, DK_, NT_)                                                         \
-    if (a.g.dv == D_ && a.g.d == DK_ && a.g.NT == NT_) {                                       \
-        auto k_rows = gather_pv_kernel<D_, DK_, NT_, false>;                                   \
-        auto k_parts = gather_pv_kernel<D_, DK_, NT_, true>;                                   \
+    if (gather_smem_bytes(a.max_lists) > static_cast<size_t>(kGatherMaxSmem) || a.cmb.parts != a.parts)
+        return cudaErrorInvalidValue;
+    const bool staged = gather_staged(a.g);
+    const size_t smem = gather_total_smem(a.max_lists, staged);
+#define SAGA_GATHER_CASE(D_, DK_, NT_, ST_)                                                    \
+    if (a.g.dv == D_ && a.g.d == DK_ && a.g.NT == NT_ && staged == ST_) {                      \
+        auto k_rows = gather_pv_kernel<D_, DK_, NT_, false, ST_>;                              \
+        auto k_parts = gather_pv_kernel<D_, DK_, NT_, true, ST_>;                              \
         auto kern = a.part_major ? k_parts : k_rows;                                           \
-        const cudaError_t attr = allow_dynamic_smem(kern, kGatherMaxSmem);                     \
+        const cudaError_t attr = allow_dynamic_smem(kern, static_cast<int>(smem));            \
         if (attr != cudaSuccess) return attr;                                                  \
         return launch_dependent(kern, grid, dim3(kThreads), smem, stream, a);                  \
     }
-    SAGA_GATHER_CASE(64, 64, 1)
-    SAGA_GATHER_CASE(64, 64, 2)
-    SAGA_GATHER_CASE(128, 128, 1)
-    SAGA_GATHER_CASE(128, 128, 2)
-    SAGA_GATHER_CASE(64, 32, 1)
-    SAGA_GATHER_CASE(64, 32, 2)
+    SAGA_GATHER_CASE(64, 64, 1, false)
+    SAGA_GATHER_CASE(64, 64, 2, false)
+    SAGA_GATHER_CASE(64, 64, 1, true)
+    SAGA_GATHER_CASE(64, 64, 2, true)
+    SAGA_GATHER_CASE(128, 128, 1, false)
+    SAGA_GATHER_CASE(128, 128, 2, false)
+    SAGA_GATHER_CASE(64, 32, 1, false)
+    SAGA_GATHER_CASE(64, 32, 2, false)
+    SAGA_GATHER_CASE(64, 32, 1, true)
+    SAGA_GATHER_CASE(64, 32, 2, true)
 #undef SAGA_GATHER_CASE
     return cudaErrorInvalidValue;
 }

@@ -28,7 +28,7 @@ SHAPES = [
     ("gqa_hk8", 1, 8, 8, 8, 64, 777, 9),
     ("narrow_keys", 2, 16, 2, 8, 32, 2500, 60),
     ("one_row_long", 1, 32, 4, 8, 64, 70000, 900),   # few long rows: the fused decode after the refresh
-    ("rows_long", 3, 32, 4, 8, 64, 70000, 900),      # several radix chunks per row
+    ("rows_long", 4, 32, 4, 8, 64, 70000, 900),      # several radix chunks per row; staged gather
     ("ragged_long", 2, 40, 4, 8, 64, 20001, 300),    # several chunks, rows not 16-byte aligned
     ("short", 3, 8, 2, 4, 64, 65, 1),
     ("N_is_l_minus_1", 1, 8, 2, 4, 64, 300, 299),
