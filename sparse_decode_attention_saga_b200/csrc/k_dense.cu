@@ -88,10 +88,24 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
                 const int z = bb * g.l_cap + tl * g.P;
                 mbar_arrive_expect_tx(&full[st], stage_bytes);
                 uint8_t* dst = smem + static_cast<size_t>(st) * stage_bytes;
-                for (int kh = 0; kh < g.hk; ++kh)
-                    for (int dh = 0; dh < KTile<D>::NBOX; ++dh)
-                        tma_load_3d(dst + (kh * KTile<D>::NBOX + dh) * g.P * KTile<D>::ROWB, &kmap,
-                                    &full[st], dh * 64, kh / a.k_group, z);
+                // key head kh of the geometry reads cache key head kh / k_group
+                // (a counter: a division here sits on the ring's turnaround)
+                if (a.k_group == 1) {
+                    for (int kh = 0; kh < g.hk; ++kh)
+                        for (int dh = 0; dh < KTile<D>::NBOX; ++dh)
+                            tma_load_3d(dst + (kh * KTile<D>::NBOX + dh) * g.P * KTile<D>::ROWB, &kmap,
+                                        &full[st], dh * 64, kh, z);
+                } else {
+                    for (int kh = 0, src = 0, r = 0; kh < g.hk; ++kh) {
+                        for (int dh = 0; dh < KTile<D>::NBOX; ++dh)
+                            tma_load_3d(dst + (kh * KTile<D>::NBOX + dh) * g.P * KTile<D>::ROWB, &kmap,
+                                        &full[st], dh * 64, src, z);
+                        if (++r == a.k_group) {
+                            r = 0;
+                            ++src;
+                        }
+                    }
+                }
                 for (int vh = 0; vh < g.hv; ++vh)
                     for (int dh = 0; dh < DVH; ++dh)
                         tma_load_3d(dst + kStageBytes + (vh * DVH + dh) * g.P * 128, &vmap,
