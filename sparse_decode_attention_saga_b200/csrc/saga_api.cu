@@ -216,6 +216,9 @@ constexpr int kPartMajorParts = 16;
 // A decode step given stored logits streams K instead when it has at most
 // this many rows of at least this many positions.
 constexpr long long kFusedFewRows = 64;
+// Static shared memory of the candidate compaction kernel (its last-digit
+// histogram and block-scan scratch), beside the row bitmap.
+constexpr size_t kCandStaticSmem = 8 * 1024;
 constexpr int kFusedMinPositions = 65536;
 // Up to this many rows per SM the compare/compact kernel reads 16 logits per
 // thread per sub-round (more bytes in flight per CTA; two CTAs per SM by its
@@ -628,7 +631,7 @@ int saga_atopn_refresh_step(const saga_dims* dims, int32_t N, const void* q, con
     // every entry kept, or a row whose bitmap does not fit on chip: the
     // compaction reads the stored logits
     const bool from_candidates = N < g.l && !few_long_rows &&
-                                 cand_select_smem(g.l) <= static_cast<size_t>(dev.max_smem);
+                                 cand_select_smem(g.l) + kCandStaticSmem <= static_cast<size_t>(dev.max_smem);
     if ((st = refresh_impl(g, dev, N, q, k, nullptr, nullptr, thresh_out, ws, s, from_candidates)))
         return st;
     if (!from_candidates) {

@@ -113,6 +113,29 @@ def test_pointer_and_workspace_validation(lib):
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+@pytest.mark.parametrize("hq,hk,hv,d,dv", [
+    (16, 1, 8, 64, 64),    # SAGA (1, 8): one key head per value head in the dense kernel
+    (16, 2, 8, 32, 64),    # Sigma-style 32-dim keys, h_v = 4 h_k
+    (16, 4, 8, 32, 64),    # h_v = 2 h_k whose stage (value rows 4x the keys) would not fit twice
+    (32, 8, 8, 64, 64),    # dense GQA
+])
+def test_dense_layouts_pass_validation(lib, hq, hk, hv, d, dv):
+    """Every SAGA layout the kernels take is a valid dense call: with no
+    device the call gets as far as the device check (arguments, shape and
+    workspace size accepted); a workspace too small for the dense kernel's
+    own geometry is refused before anything runs."""
+    dd = _lib.dims(2, hq, hk, hv, d, 3000, 3000, dv)
+    need = _lib.workspace_bytes(dd, 8)
+    assert need > 0
+    big = _ws(need + 512)
+    base = (big.data_ptr() + 255) // 256 * 256
+    st = lib.saga_decode_dense(ctypes.byref(dd), 16, 16, 16, 16, base, need, None)
+    assert st in (_lib.SAGA_ERR_DEVICE, _lib.SAGA_ERR_CUDA)
+    assert lib.saga_decode_dense(ctypes.byref(dd), 16, 16, 16, 16, base, 256, None) == \
+        _lib.SAGA_ERR_WORKSPACE
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_a_device_reports_no_device(lib):
     d = _lib.dims(1, 4, 1, 2, 64, 64)
     need = _lib.workspace_bytes(d, 8)
