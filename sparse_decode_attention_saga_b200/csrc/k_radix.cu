@@ -31,7 +31,9 @@ namespace saga {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarpsR = kThreads / 32;
 constexpr int kLoads = 16;
+constexpr int kMemberBuf = 64;  // pass 1: members a warp lists at a time
 
 // Block-wide exclusive scan of one value per thread; returns the block total.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t& excl,
@@ -72,6 +74,8 @@ __global__ void __launch_bounds__(kThreads, VEC == 4 ? 8 : 4) radix_pass_kernel(
     __shared__ uint32_t warp_tot[kThreads / 32];
     __shared__ int is_last;
     __shared__ int s_cand;  // pass 1: candidates this CTA has copied out
+    // pass 1: each warp's members of the round (positions), kMemberBuf at a time
+    __shared__ int s_members[PASS == 1 ? kWarpsR * kMemberBuf : 1];
 
     pdl_wait();  // logits, histograms and the previous pass's state
     pdl_trigger();
@@ -83,6 +87,7 @@ __global__ void __launch_bounds__(kThreads, VEC == 4 ? 8 : 4) radix_pass_kernel(
     const uint32_t prefix = PASS == 0 ? 0u : __ldcg(a.state + row * 2);
     __syncthreads();
     const bool from_cand = PASS == 2 && a.cand != nullptr;
+    const int lane = tid & 31, warp = tid >> 5;
 
     const float* src = a.logits + row * a.l;
     const int per = radix_chunk_len(a.l, a.chunks);
@@ -100,13 +105,6 @@ __global__ void __launch_bounds__(kThreads, VEC == 4 ? 8 : 4) radix_pass_kernel(
     // would take its key's place in pass 0 but not in this compare.)
     const float lo_f = key_to_float(prefix << 21);
     const bool all_members = isnan(lo_f);
-    // the member's key into the histogram (its bucket's next digit) and, with
-    // a candidate buffer, its (position, logit) into this chunk's part
-    auto member = [&](float x, int j) {
-        const uint32_t key = float_to_key(x);
-        if ((key >> high) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-        if (cdst) cdst[atomicAdd(&s_cand, 1)] = make_int2(j, __float_as_int(x));
-    };
     // 64 bytes of independent coalesced loads per thread per round (16-byte
     // loads when the rows are 16-byte aligned) keep enough bytes in flight to
     // stream the logits at HBM speed; whole rounds skip the bounds checks.
@@ -128,8 +126,7 @@ __global__ void __launch_bounds__(kThreads, VEC == 4 ? 8 : 4) radix_pass_kernel(
         }
         if constexpr (PASS == 1) {
             // Members are a few percent of the logits: a bitmask of this
-            // thread's members (branch-free), then one short loop over the
-            // set bits, each member's logit read again from L1.
+            // thread's members (branch-free) first.
             uint32_t m = 0u;
 #pragma unroll
             for (int k = 0; k < kLoadsV; ++k)
@@ -139,11 +136,42 @@ __global__ void __launch_bounds__(kThreads, VEC == 4 ? 8 : 4) radix_pass_kernel(
                     const bool in = (kWhole || j < j1) && (v[k][c] >= lo_f || all_members);
                     m |= static_cast<uint32_t>(in) << (k * VEC + c);
                 }
-            while (m) {
-                const int e = __ffs(m) - 1;
-                m &= m - 1u;
-                const int j = base + ((e / VEC) * kThreads + tid) * VEC + e % VEC;
-                member(__ldg(src + j), j);
+            // The warp's members of the round in one list (a warp scan of the
+            // per-thread counts; positions only), then one pass of the warp's
+            // lanes over the list: each member's logit read again (L2), its
+            // key into the histogram, and the candidates stored together.
+            const int cnt_t = __popc(m);
+            int incl = cnt_t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += x;
+            }
+            const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+            if (wtot) {
+                int* wbuf = s_members + warp * kMemberBuf;
+                int wbase = 0;
+                if (cdst && lane == 0) wbase = atomicAdd(&s_cand, wtot);
+                wbase = __shfl_sync(0xffffffffu, wbase, 0);
+                // (more members than the buffer holds: several batches)
+                for (int b0 = 0; b0 < wtot; b0 += kMemberBuf) {
+                    int at = incl - cnt_t;
+                    for (uint32_t mm = m; mm; mm &= mm - 1u, ++at) {
+                        const int e = __ffs(mm) - 1;
+                        if (at >= b0 && at < b0 + kMemberBuf)
+                            wbuf[at - b0] = base + ((e / VEC) * kThreads + tid) * VEC + e % VEC;
+                    }
+                    __syncwarp();
+                    const int nbatch = min(kMemberBuf, wtot - b0);
+                    for (int i = lane; i < nbatch; i += 32) {
+                        const int j = wbuf[i];
+                        const float x = __ldg(src + j);
+                        const uint32_t key = float_to_key(x);
+                        if ((key >> high) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+                        if (cdst) cdst[wbase + b0 + i] = make_int2(j, __float_as_int(x));
+                    }
+                    __syncwarp();
+                }
             }
         } else {
 #pragma unroll
