@@ -220,22 +220,26 @@ __global__ void __launch_bounds__(kThreads) lists_to_index_kernel(const IndexArg
 }
 
 // One CTA per row over the radix candidates.  With the radix state of the
-// first two digits (a.state), the threshold's last digit comes first: the
-// candidates in the 22-bit prefix bucket are histogrammed by their last 10
-// bits in shared memory and a block scan picks the bin holding the rank
+// first two digits (a.state) the threshold's 22-bit prefix is known: one
+// pass over the candidates sets the bit of every position above that bucket
+// in a shared bitmap of the row (kept whatever the last digit), counts the
+// bucket's candidates by their last 10 bits in a shared histogram and
+// stashes them (a few per row); a block scan picks the bin holding the rank
 // still sought, which completes the exact N-th largest logit (written to
-// a.thresh; the third radix pass is not needed).  Then every candidate at or
-// above the threshold sets its position's bit in a shared bitmap (a
-// position is a candidate at most once), each thread takes a contiguous run
-// of bitmap words and a block scan of the runs' counts gives every word's
-// rank, and each kept candidate is written at its word's rank plus the set
-// bits below it, so the output is ascending whatever order the candidates
-// came in.  The row's largest logit is the largest candidate.  Nothing kept
-// (only when the threshold lies above every logit) keeps the row's maxima,
-// as the compaction over stored logits does.
+// a.thresh; the third radix pass is not needed), and only the stashed
+// candidates are compared with it.  Without the state the thresholds are
+// given and every candidate is compared.  Then each thread takes a
+// contiguous run of bitmap words, a block scan of the runs' counts gives
+// every word's rank, and each kept candidate is written at its word's rank
+// plus the set bits below it, so the output is ascending whatever order the
+// candidates came in (a position is a candidate at most once).  The row's
+// largest logit is the largest candidate.  Nothing kept (only when the
+// threshold lies above every logit) keeps the row's maxima, as the
+// compaction over stored logits does.
 // Dynamic shared memory (cand_select_smem): bitmap [words] | word ranks [words].
 constexpr int kCandThreads = 512;
 constexpr int kCandWarps = kCandThreads / 32;
+constexpr int kCandStash = 1024;
 
 __device__ __forceinline__ uint32_t cand_block_scan(uint32_t v, uint32_t& excl, uint32_t* warp_tot) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -263,6 +267,8 @@ __global__ void __launch_bounds__(kCandThreads) cand_select_kernel(const CandSel
     __shared__ float red[kCandWarps];
     __shared__ uint32_t hist[1024];
     __shared__ float s_tau;
+    __shared__ int s_nstash;
+    __shared__ int2 stash[kCandStash];  // the candidates of the threshold's 22-bit bucket
     pdl_wait();  // candidates and radix state (or thresholds) from the radix passes
     pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -295,15 +301,32 @@ __global__ void __launch_bounds__(kCandThreads) cand_select_kernel(const CandSel
         }
     };
 
+    // Kept bits: with the radix state the row's 22-bit threshold prefix is
+    // known, so one pass sets the bit of every candidate above that bucket
+    // (kept whatever the last digit), counts the bucket's candidates by their
+    // last 10 bits and stashes them; the digit holding the rank gives the
+    // threshold, and only the stashed ones are compared with it (a second
+    // pass over the candidates only when the bucket overflows the stash).
     float tau;
+    float m = -kInf;
+    for (int w = tid; w < words; w += kCandThreads) bm[w] = 0u;
     if (a.state) {
-        // the last 10 bits of the N-th largest key
-        const uint32_t prefix = __ldcg(a.state + row * 2), rank = __ldcg(a.state + row * 2 + 1);
         for (int i = tid; i < 1024; i += kCandThreads) hist[i] = 0u;
-        __syncthreads();
-        each([&](int, float x) {
+        if (tid == 0) s_nstash = 0;
+    }
+    __syncthreads();
+    if (a.state) {
+        const uint32_t prefix = __ldcg(a.state + row * 2), rank = __ldcg(a.state + row * 2 + 1);
+        each([&](int pos, float x) {
+            m = fmaxf(m, x);
             const uint32_t key = float_to_key(x);
-            if ((key >> 10) == prefix) atomicAdd(&hist[key & 1023u], 1u);
+            if ((key >> 10) > prefix) {
+                atomicOr(bm + (pos >> 5), 1u << (pos & 31));
+            } else if ((key >> 10) == prefix) {
+                atomicAdd(&hist[key & 1023u], 1u);
+                const int at = atomicAdd(&s_nstash, 1);
+                if (at < kCandStash) stash[at] = make_int2(pos, __float_as_int(x));
+            }
         });
         __syncthreads();
         constexpr int kPer = 1024 / kCandThreads;  // bins per thread, from the top
@@ -333,26 +356,37 @@ __global__ void __launch_bounds__(kCandThreads) cand_select_kernel(const CandSel
         }
         __syncthreads();
         tau = s_tau;
+        const int nst = s_nstash;
+        if (nst <= kCandStash) {
+            for (int i = tid; i < nst; i += kCandThreads) {
+                const int2 p = stash[i];
+                if (__int_as_float(p.y) >= tau) atomicOr(bm + (p.x >> 5), 1u << (p.x & 31));
+            }
+        } else {
+            each([&](int pos, float x) {
+                if ((float_to_key(x) >> 10) == prefix && x >= tau) atomicOr(bm + (pos >> 5), 1u << (pos & 31));
+            });
+        }
     } else {
         tau = __ldg(a.thresh + row);
-    }
-
-    float m = -kInf;
-    uint32_t total = 0;
-    for (int pass = 0; pass < 2; ++pass) {
-        for (int w = tid; w < words; w += kCandThreads) bm[w] = 0u;
-        __syncthreads();
         each([&](int pos, float x) {
-            if (pass == 0) m = fmaxf(m, x);
+            m = fmaxf(m, x);
             if (x >= tau) atomicOr(bm + (pos >> 5), 1u << (pos & 31));
         });
-        if (pass == 0) {
-            m = warp_max(m);
-            if (lane == 0) red[warp] = m;
-        }
-        __syncthreads();
-        const int run = (words + kCandThreads - 1) / kCandThreads;
-        const int w0 = min(words, tid * run), w1 = min(words, w0 + run);
+    }
+    m = warp_max(m);
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    m = red[0];
+#pragma unroll
+    for (int w = 1; w < kCandWarps; ++w) m = fmaxf(m, red[w]);
+
+    // word ranks; nothing kept (only when the threshold lies above every
+    // logit) keeps the row's maxima, as the compaction over stored logits does
+    const int run = (words + kCandThreads - 1) / kCandThreads;
+    const int w0 = min(words, tid * run), w1 = min(words, w0 + run);
+    uint32_t total = 0;
+    for (int pass = 0; pass < 2; ++pass) {
         uint32_t c = 0;
         for (int w = w0; w < w1; ++w) c += __popc(bm[w]);
         uint32_t at;
@@ -361,14 +395,12 @@ __global__ void __launch_bounds__(kCandThreads) cand_select_kernel(const CandSel
             wrank[w] = at;
             at += __popc(bm[w]);
         }
-        if (pass == 0) {
-            m = red[0];
-#pragma unroll
-            for (int w = 1; w < kCandWarps; ++w) m = fmaxf(m, red[w]);
-        }
-        if (total > 0) break;
-        tau = m;  // nothing passed: keep the maxima
+        if (total > 0 || pass == 1) break;
         if (tid == 0 && a.empty_rows) atomicAdd(a.empty_rows, 1u);
+        __syncthreads();
+        each([&](int pos, float x) {
+            if (x >= m) atomicOr(bm + (pos >> 5), 1u << (pos & 31));
+        });
         __syncthreads();
     }
     __syncthreads();

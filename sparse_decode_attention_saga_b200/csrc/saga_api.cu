@@ -217,8 +217,9 @@ constexpr int kPartMajorParts = 16;
 // this many rows of at least this many positions.
 constexpr long long kFusedFewRows = 64;
 // Static shared memory of the candidate compaction kernel (its last-digit
-// histogram and block-scan scratch), beside the row bitmap.
-constexpr size_t kCandStaticSmem = 8 * 1024;
+// histogram, the stash of its threshold bucket's candidates and block-scan
+// scratch), beside the row bitmap.
+constexpr size_t kCandStaticSmem = 16 * 1024;
 constexpr int kFusedMinPositions = 65536;
 // Up to this many rows per SM the compare/compact kernel reads 16 logits per
 // thread per sub-round (more bytes in flight per CTA; two CTAs per SM by its
