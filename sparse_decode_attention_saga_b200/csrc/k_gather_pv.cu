@@ -7,7 +7,7 @@
 // Key Contributions #3).
 //
 // A row's kept entries live in one or more ascending lists of (position,
-// logit) pairs: one contiguous list from the compare/compact kernel
+// logit) pairs: one contiguous list from a compaction kernel
 // (kListContiguous), or one list per
 // (streaming CTA slot, consumer warp) from the fused kernel (kListSegments).
 // Grid (parts, rows), or (rows, parts) with part_major: every CTA builds the
@@ -19,11 +19,12 @@
 // row and no row waits for a second wave of CTAs that turn out to be empty.
 // Each warp then works through its own contiguous part of that share without
 // block barriers: 32 entries at a time, one (position, logit) per lane read
-// with coalesced loads, the 32 value rows copied with cp.async into a
-// two-stage per-warp ring in shared memory (the next 32 rows' loads in
-// flight while these are summed), and each row read back by a lane group
-// (8 or 16 lanes, 16 bytes each), weighted by exp(s - m) and accumulated in
-// fp32.  m is the row's largest logit, which is always kept when anything is
+// with coalesced loads, and each value row handled by a lane group (8 or 16
+// lanes, 16 bytes each), weighted by exp(s - m) and accumulated in fp32.
+// With long rows and many of them (STAGED) the 32 value rows are copied
+// with cp.async into a two-stage per-warp ring in shared memory (the next
+// 32 rows' loads in flight while these are summed); otherwise they are
+// loaded into registers, a few per lane at a time.  m is the row's largest logit, which is always kept when anything is
 // (tau_eff <= max), so no running max is needed.  The share's (m, sum of
 // weights, count, row max, unnormalised output) record is merged across
 // shares by the last CTA of the row; all shares used the same reference m,

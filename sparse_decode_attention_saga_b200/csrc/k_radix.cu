@@ -16,11 +16,13 @@
 // (prefix, rank) for the next pass, or the threshold after the last pass.
 // No CTA waits for another.  With a candidate buffer, pass 1 also copies the
 // (position, logit) of every key at or above the lower edge of pass 0's
-// bucket into its chunk's part of the buffer (one shared-memory counter per
-// CTA; the order inside a chunk is not fixed), and pass 2 reads only those
-// candidates, each CTA its own chunk's.  The kept set (logit >= threshold)
-// lies among them, so the ordered compaction can read them instead of the
-// logits (k_select.cu).
+// bucket into its chunk's part of the buffer (each warp lists a round's
+// members in shared memory and stores them together at a place reserved
+// from a per-CTA counter; the order inside a chunk is not fixed), and pass 2
+// reads only those candidates, each CTA its own chunk's.  The kept set
+// (logit >= threshold) lies among them, so a refresh step stops after pass
+// 1 and one kernel finds the last digit and compacts the kept entries from
+// the candidates alone (k_select.cu).
 #include <type_traits>
 
 #include "saga_device.cuh"
