@@ -47,7 +47,9 @@
  *     16-byte aligned), the thresholds and the workspace included.  The
  *     library allocates no device memory.
  *   - Asynchrony: every call only enqueues work on `stream` and returns; no
- *     call synchronises the host or reads device data back.  All grids are
+ *     call synchronises the host or reads device data back (except the two
+ *     workspace readers, saga_workspace_error and saga_workspace_empty_rows,
+ *     which say so).  All grids are
  *     sized from the shapes, never from data, so a sequence of calls can be
  *     captured in a CUDA graph (make one uncaptured call per shape first so
  *     device properties are cached outside the capture).
