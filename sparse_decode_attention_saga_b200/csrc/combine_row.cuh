@@ -23,6 +23,11 @@ namespace saga {
 
 constexpr int kCombineThreads = 256;
 
+// The empty-set rule's row, by one warp: the positions whose logit equals
+// the row maximum m_star (recomputed bit for bit with the streaming
+// kernel's tensor-core routine), their count, and the mean of their value
+// rows into out_row.  With the fused kernel's per-list maxima (a.seg_mall)
+// only the lists holding m_star are recomputed, otherwise the whole row.
 // raw: out_row gets the sum of the value rows at m_star instead of their
 // mean.  idx_out (nullable): their positions, ascending.  Returns their
 // number (all lanes).
@@ -48,7 +53,9 @@ __device__ int fallback_row(const CombineArgs& a, long long row, float m_star, f
 #pragma unroll
     for (int c = 0; c < CPL; ++c) osum[c] = 0.f;
     int count = 0;
-    for (int j0 = 0; j0 < g.l; j0 += 16) {
+    // positions j0 .. j0+15: their logits recomputed, those equal to m_star
+    // (ascending: h, then lane) counted and their value rows summed
+    auto block = [&](int j0) {
         // 16 key rows of head kh into the swizzled tile layout of qk_mma
         for (int q8 = lane; q8 < 16 * D / 8; q8 += 32) {
             const int r = q8 / (D / 8), cc = q8 - r * (D / 8);
@@ -80,7 +87,7 @@ __device__ int fallback_row(const CombineArgs& a, long long row, float m_star, f
                 const int src = __ffs(ball) - 1;
                 ball &= ball - 1;
                 const int pos = j0 + (src >> 2) + 8 * h;
-                if (idx_out && lane == 0) idx_out[count] = pos;  // ascending: h, then lane
+                if (idx_out && lane == 0) idx_out[count] = pos;
                 const __nv_bfloat16* vr =
                     V + ((static_cast<size_t>(bb) * g.l_cap + pos) * g.hv + vh) * DV + lane * CPL;
 #pragma unroll
@@ -88,6 +95,33 @@ __device__ int fallback_row(const CombineArgs& a, long long row, float m_star, f
                 ++count;
             }
         }
+    };
+    if (a.seg_mall) {
+        // The fused kernel's per-(slot, warp) maxima say which of its lists
+        // hold the row maximum: only their positions are recomputed (for each
+        // slot in order, its tiles in order, in each tile the warps' 16-row
+        // blocks in order, so positions stay ascending).
+        const long long T = static_cast<long long>(g.b) * g.tiles;
+        const long long x0 = static_cast<long long>(bb) * g.tiles;
+        const int c_first = cta_of_tile(x0, T, a.C);
+        const int slots = cta_of_tile(x0 + g.tiles - 1, T, a.C) - c_first + 1;
+        const float* mall_row = a.seg_mall + static_cast<size_t>(row) * g.S_cap * g.WPK;
+        for (int sl = 0; sl < slots; ++sl) {
+            const uint32_t subs =
+                __ballot_sync(0xffffffffu, lane < g.WPK && __ldcg(mall_row + sl * g.WPK + lane) == m_star);
+            if (!subs) continue;
+            const int c = c_first + sl;
+            const long long t0 = cta_tile_begin(T, a.C, c), t1 = cta_tile_begin(T, a.C, c + 1);
+            const long long s0 = t0 > x0 ? t0 : x0, s1 = t1 < x0 + g.tiles ? t1 : x0 + g.tiles;
+            for (long long t = s0; t < s1; ++t)
+                for (uint32_t sm = subs; sm; sm &= sm - 1u) {
+                    const int sub = __ffs(sm) - 1;
+                    for (int mbi = 0; mbi < g.MBW; ++mbi)
+                        block(static_cast<int>((t - x0) * g.P) + (sub * g.MBW + mbi) * 16);
+                }
+        }
+    } else {
+        for (int j0 = 0; j0 < g.l; j0 += 16) block(j0);
     }
 #pragma unroll
     for (int c = 0; c < CPL; ++c) out_row[lane * CPL + c] = raw ? osum[c] : osum[c] / static_cast<float>(count);

@@ -584,6 +584,8 @@ static int atopn_decode_impl(const saga_dims* dims, const void* q, const void* k
     ga.cmb.sel_cnt = sel_cnt;
     ga.cmb.sel_idx = sel_idx;
     ga.cmb.empty_rows = part ? nullptr : ws_empty_rows(ws, L);
+    ga.cmb.C = a.C;              // the fallback recomputes only the lists
+    ga.cmb.seg_mall = a.seg_mall;  // that hold the row maximum
     g_launches += 1;
     if ((e = launch_gather_pv(ga, s)) != cudaSuccess || !sel_idx) return cuda_status(e);
 

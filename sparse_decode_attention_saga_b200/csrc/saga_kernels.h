@@ -187,6 +187,10 @@ struct CombineArgs {
     // Optional: counts the rows that kept nothing and took the empty-set
     // fallback (one atomic add per such row; not for a shard's partials).
     uint32_t* empty_rows;
+    // Optional, with the fused kernel's lists (C its grid): the per-(slot,
+    // warp) maxima [rows][S_cap][WPK], so that the fallback recomputes only
+    // the lists that hold the row maximum.
+    const float* seg_mall;
 };
 // Gathered softmax-PV over kept lists -> partial records.
 enum ListMode : int {
