@@ -96,7 +96,12 @@ __device__ int fallback_row(const CombineArgs& a, long long row, float m_star, f
             }
         }
     };
-    if (a.seg_mall) {
+    // (64-dim values with at most 8 query heads per key head only: in the
+    // other instantiations the extra loop state spills registers of the
+    // gather kernel that inlines this)
+    bool lists_only = false;
+    if constexpr (DV == 64 && NT == 1) lists_only = a.seg_mall != nullptr;
+    if (lists_only) {
         // The fused kernel's per-(slot, warp) maxima say which of its lists
         // hold the row maximum: only their positions are recomputed (for each
         // slot in order, its tiles in order, in each tile the warps' 16-row
@@ -110,14 +115,15 @@ __device__ int fallback_row(const CombineArgs& a, long long row, float m_star, f
             const uint32_t subs =
                 __ballot_sync(0xffffffffu, lane < g.WPK && __ldcg(mall_row + sl * g.WPK + lane) == m_star);
             if (!subs) continue;
+            // the slot's tiles of this batch row, as offsets in the row
             const int c = c_first + sl;
-            const long long t0 = cta_tile_begin(T, a.C, c), t1 = cta_tile_begin(T, a.C, c + 1);
-            const long long s0 = t0 > x0 ? t0 : x0, s1 = t1 < x0 + g.tiles ? t1 : x0 + g.tiles;
-            for (long long t = s0; t < s1; ++t)
+            const int r0 = static_cast<int>(max(cta_tile_begin(T, a.C, c) - x0, 0ll));
+            const int r1 = static_cast<int>(min(cta_tile_begin(T, a.C, c + 1) - x0,
+                                                static_cast<long long>(g.tiles)));
+            for (int tl = r0; tl < r1; ++tl)
                 for (uint32_t sm = subs; sm; sm &= sm - 1u) {
                     const int sub = __ffs(sm) - 1;
-                    for (int mbi = 0; mbi < g.MBW; ++mbi)
-                        block(static_cast<int>((t - x0) * g.P) + (sub * g.MBW + mbi) * 16);
+                    for (int mbi = 0; mbi < g.MBW; ++mbi) block(tl * g.P + (sub * g.MBW + mbi) * 16);
                 }
         }
     } else {
