@@ -51,7 +51,7 @@ def _growth_loop(w: Workload, seed: int):
         assert_mask_exact(dec, qs[t], K, idx, cnt, what=f"t={t}")
         assert_mask_within_band(mask_gpu, m_ref, s_ref, tau_ref, f"t={t}")
         ref = oracle.attend_masked(s_ref, mask_gpu, Vh)
-        assert_outputs_close(out_l.cpu().numpy(), ref, f"t={t} stored-logits")
+        assert_outputs_close(out_l.cpu().numpy(), ref, f"t={t} with positions")
         assert_outputs_close(out_f.cpu().numpy(), ref, f"t={t} fused")
     return dec
 

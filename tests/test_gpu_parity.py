@@ -192,8 +192,9 @@ def run_loop_and_compare(w, seed=0, gen_device="cuda", rows=None):
     """Steps 0..steps-1 on the GPU and in the oracle; returns the number of
     in-band mask flips.  Each step runs twice: without and with the kept
     positions emitted.  On reuse steps both runs take the fused path (the
-    on-chip compare of the streaming kernel), on refresh steps the
-    stored-logits path; either way the emitted mask is checked bit for bit
+    on-chip compare of the streaming kernel), on refresh steps the one-call
+    refresh step (its candidate compaction); either way the emitted mask is
+    checked bit for bit
     against the oracle's selection over the GPU's own logits, and against
     the oracle's end-to-end step within the band."""
     qs, K, V = device_inputs(w, seed, gen_device=gen_device)
@@ -220,7 +221,7 @@ def run_loop_and_compare(w, seed=0, gen_device="cuda", rows=None):
         assert_mask_exact(dec, qs[t], K, idx, cnt, b_sel, f"t={t}")
         flips += assert_mask_within_band(mask_gpu, m_ref, s_ref, tau_ref, f"t={t}")
         ref = oracle.attend_masked(s_ref, mask_gpu, Vh)
-        assert_outputs_close(out_l[b_sel].cpu().numpy(), ref, f"t={t} stored-logits")
+        assert_outputs_close(out_l[b_sel].cpu().numpy(), ref, f"t={t} with positions")
         assert_outputs_close(out_fused[b_sel].cpu().numpy(), ref, f"t={t} fused")
     return flips
 
@@ -293,8 +294,8 @@ def test_zero_query_and_unit_values():
 def test_same_query_reuse_keeps_the_refresh_mask():
     """A reuse step with the refresh step's own query keeps exactly the
     refresh step's set: the fused on-chip compare (reuse) against the
-    stored-logits compare (refresh).  The outputs sum the same entries in a
-    different order, so they agree to rounding."""
+    refresh step's compaction of its candidates.  The outputs sum the same
+    entries in a different order, so they agree to rounding."""
     w = wl("same", 2, 32, 4, 8, 64, 5000, None, N=100, n=4, steps=1)
     qs, K, V = device_inputs(w, seed=11, steps=1)
     dec = AtopNDecoder.for_workload(w)
