@@ -4,16 +4,20 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
                     [--impl ours|reference]
 
-A step is one decode token of the Atop-N loop: refresh (exact radix select of
-the N-th largest logit) when t mod n == 0, otherwise the fused reuse step,
-always followed by the kept-entry softmax and gathered value sum.  Warm-up
-runs steps 0..W-1; the timed region runs steps W..W+K-1 as one CUDA-graph
-replay (the pages time their decode loop as captured CUDA graphs), timed
-with CUDA events on the capture stream, max over ranks.  Inputs (K and V
-caches of 3 GB at the default workload) are larger than the 126 MB L2, so
-no flush is needed between steps; caches under 4x L2 are timed one graph per
-step with an L2 flush between.  The end-to-end leg runs the same steps
-through AtopNDecoder.host_loop (queries from, outputs to pinned host memory).
+A step is one decode token of the Atop-N loop: the refresh step (exact radix
+select of the N-th largest logit, then the decode with it) when t mod n == 0,
+otherwise the fused reuse step, always followed by the kept-entry softmax and
+gathered value sum.  Warm-up runs steps 0..W-1; the timed region runs steps
+W..W+K-1 as one CUDA-graph replay (the pages time their decode loop as
+captured CUDA graphs), timed with CUDA events on the capture stream, max over
+ranks, and reported as `window`.  The headline value is the schedule's mix,
+one refresh step and n - 1 reuse steps per n tokens, each kind timed as
+CUDA-graph replays in the same run, so that it does not depend on where the
+window falls in the refresh period.  Inputs (K and V caches of 3 GB at the
+default workload) are larger than the 126 MB L2, so no flush is needed
+between steps; caches under 4x L2 are timed one graph per step with an L2
+flush between.  The end-to-end leg runs whole refresh periods through
+AtopNDecoder.host_loop (queries from, outputs to pinned host memory).
 
 Prints ONE JSON line (rank 0).  N > 1 runs independent replicas (one batch
 per GPU, no collective on the data path; weak scaling).
