@@ -328,6 +328,9 @@ __global__ void __launch_bounds__(kCandThreads) cand_select_kernel(const CandSel
                 if (at < kCandStash) stash[at] = make_int2(pos, __float_as_int(x));
             }
         });
+        // (the bucket's lower edge stands if no bin holds the rank, which the
+        // radix state of finite logits rules out)
+        if (tid == 0) s_tau = key_to_float(prefix << 10);
         __syncthreads();
         constexpr int kPer = 1024 / kCandThreads;  // bins per thread, from the top
         const int top = 1024 - tid * kPer;
