@@ -127,7 +127,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // ----------------------------------------------------------------- TMA
 
 // 3-D tiled bulk tensor load global -> shared, completion counted in bytes on
-// `bar`.  No multicast.  x is the innermost coordinate (elements).
+// `bar`, into this CTA's shared memory only.  x is the innermost coordinate
+// (elements).
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y, int z) {
     asm volatile(
